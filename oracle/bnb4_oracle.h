@@ -1,0 +1,88 @@
+/*
+ * bnb4_oracle.h -- plain, slow CPU oracle for 4-bit blockwise weight
+ * quantization (NF4 / FP4) and the matmuls that consume it.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This header and bnb4_oracle.c are used by the
+ * test suite, by the smoke check and by the benchmark's CPU-baseline leg.
+ * The product library (libbnb4.so) neither includes nor links anything in
+ * this directory, and this directory includes nothing from the product.
+ *
+ * Every function is single-threaded, uses no blocking or reordering, and
+ * computes in the precision stated beside it.  Sources (page title, section):
+ *   - "mps-bitsandbytes 0.4.7", Features table and Functional API
+ *     (quantize_nf4 / dequantize_nf4 / matmul_nf4: per-block absmax scaling
+ *     to [-1, 1], nearest code of a 16-entry table, two codes per byte).
+ *   - "Feat/mps gemm 4bit bf16", table "What runs natively now" (the op list:
+ *     quantize_4bit, dequantize_4bit, gemv_4bit, gemm_4bit,
+ *     gemm_4bit_backward = grad_output @ dequantize_4bit(B)) and section
+ *     "Correctness" (exact nearest-code search, never through a lookup table).
+ */
+#ifndef BNB4_ORACLE_H
+#define BNB4_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* quant types and dtypes use the same numeric codes as the product ABI, but
+ * are declared here independently. */
+#define ORACLE_NF4 0
+#define ORACLE_FP4 1
+#define ORACLE_F32 0
+#define ORACLE_F16 1
+#define ORACLE_BF16 2
+
+/* 16 fp32 code values for a quant type (index order = stored nibble). */
+int oracle_code_table(int qtype, float out[16]);
+
+/* element conversions (the oracle's own, by arithmetic on the values) */
+float oracle_f16_to_f32(uint16_t h);
+float oracle_bf16_to_f32(uint16_t h);
+uint16_t oracle_f32_to_f16_rne(float f);
+uint16_t oracle_f32_to_bf16_rne(float f);
+
+/* array forms of the conversions (dtype codes as above) */
+int oracle_to_f32_array(const void *in, int dtype, int64_t n, float *out);
+int oracle_from_f32_array(const float *in, int64_t n, int dtype, void *out);
+
+/* Quantize n elements of x (dtype) in blocks of `blocksize` consecutive
+ * elements.  packed: ceil(n/2) bytes, absmax: ceil(n/blocksize) floats. */
+int oracle_quantize(const void *x, int dtype, int64_t n, int blocksize,
+                    int qtype, uint8_t *packed, float *absmax);
+
+/* out[i] = RN_dtype( fp32(code[idx_i] * absmax[i / blocksize]) ) */
+int oracle_dequantize(const uint8_t *packed, const float *absmax, int64_t n,
+                      int blocksize, int qtype, int out_dtype, void *out);
+
+/* Y[m, j] = sum_k X[m, k] * Wdeq[j, k] (+ bias[j]) in float64, where
+ * Wdeq = fp32(code * absmax) is the [N, K] weight quantized row-major as one
+ * flat array.  X is [M, K] of x_dtype; bias (nullable) is [N] of x_dtype. */
+int oracle_matmul(const void *X, int x_dtype, const uint8_t *packed,
+                  const float *absmax, const void *bias, int64_t M, int64_t N,
+                  int64_t K, int blocksize, int qtype, double *Y);
+
+/* The same product, only at `count` (m, j) positions: Y[i] = Y(ms[i], js[i]). */
+int oracle_matmul_entries(const void *X, int x_dtype, const uint8_t *packed,
+                          const float *absmax, const void *bias, int64_t M,
+                          int64_t N, int64_t K, int blocksize, int qtype,
+                          const int64_t *ms, const int64_t *js, int64_t count,
+                          double *Y);
+
+/* dX[m, k] = sum_j dY[m, j] * Wdeq[j, k] in float64. dY is [M, N] of dy_dtype. */
+int oracle_matmul_backward(const void *dY, int dy_dtype, const uint8_t *packed,
+                           const float *absmax, int64_t M, int64_t N, int64_t K,
+                           int blocksize, int qtype, double *dX);
+
+/* The backward product at `count` (m, k) positions. */
+int oracle_matmul_backward_entries(const void *dY, int dy_dtype,
+                                   const uint8_t *packed, const float *absmax,
+                                   int64_t M, int64_t N, int64_t K,
+                                   int blocksize, int qtype, const int64_t *ms,
+                                   const int64_t *ks, int64_t count, double *dX);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,98 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins catch each.
+
+Each mutation edits one line of a temporary copy of ``oracle/bnb4_oracle.c``,
+builds it on the CPU and runs the pin checks against it.  A mutation that no
+pin notices would mean the pins do not cover that step.
+"""
+import ctypes
+import os
+import shutil
+import subprocess
+import tempfile
+
+import pytest
+
+import oracle
+import test_oracle as pins  # noqa: E402  (tests/ is on sys.path under pytest)
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "bnb4_oracle.c")
+
+MUTATIONS = {
+    "ties_to_largest_index": ("if (d < bd) {", "if (d <= bd) {"),
+    "nibble_order_swapped": ("packed[i >> 1] |= (uint8_t)(idx << 4);\n            else\n                packed[i >> 1] |= (uint8_t)idx;",
+                             "packed[i >> 1] |= (uint8_t)idx;\n            else\n                packed[i >> 1] |= (uint8_t)(idx << 4);"),
+    "absmax_without_abs": ("float a = fabsf(load_elem(x, dtype, i));", "float a = load_elem(x, dtype, i);"),
+    "reciprocal_instead_of_quotient": ("load_elem(x, dtype, i) / amax;", "load_elem(x, dtype, i) * (1.0f / amax);"),
+    "zero_block_not_special": ("(amax == 0.0f) ? 0.0f : load_elem", "(0) ? 0.0f : load_elem"),
+    "dequant_operands_rounded_to_bf16": (
+        "float p = c * a;\n    return p;",
+        "float p = oracle_bf16_to_f32(oracle_f32_to_bf16_rne(c)) *"
+        " oracle_bf16_to_f32(oracle_f32_to_bf16_rne(a));\n    return p;"),
+    "dequant_skips_fp32_rounding": (
+        "store_elem(out, out_dtype, i, dequant_f32(packed, absmax, i, blocksize, code));",
+        "if (out_dtype == ORACLE_BF16) ((uint16_t *)out)[i] = encode_format(round_to_format("
+        "(double)code[code_index(packed, i)] * (double)absmax[i / blocksize], 8, -126,"
+        " ldexp(2.0 - ldexp(1.0, -7), 127)), 7, 127, -126, 255);"
+        " else store_elem(out, out_dtype, i, dequant_f32(packed, absmax, i, blocksize, code));"),
+    "fp4_exponent_bias": ("(1.0 + 0.5 * m) * ldexp(1.0, e - 1)", "(1.0 + 0.5 * m) * ldexp(1.0, e)"),
+    "nf4_literal_typo": ("-0.2844414f", "-0.2844441f"),
+    "rounding_truncates": ("double r = nearbyint(a / quantum) * quantum;", "double r = floor(a / quantum) * quantum;"),
+    "forward_weight_transposed": ("dequant_f32(packed, absmax, j * K + k, blocksize, code);\n        acc += xv * wv;",
+                                  "dequant_f32(packed, absmax, k * N + j, blocksize, code);\n        acc += xv * wv;"),
+    "forward_bias_dropped": ("acc += (double)load_elem(bias, x_dtype, j);", "acc += 0.0;"),
+    "backward_weight_transposed": ("j * K + k, blocksize, code);\n        acc += g * wv;",
+                                   "k * N + j, blocksize, code);\n        acc += g * wv;"),
+}
+
+PIN_CHECKS = [
+    lambda: pins.test_worked_example_golden(),
+    lambda: pins.test_nf4_table_matches_golden_literals_and_invariants(),
+    lambda: pins.test_fp4_table_closed_form(),
+    lambda: pins.test_special_blocks(),
+    lambda: [pins.test_ties_go_to_smallest_index(q) for q in ("nf4", "fp4")],
+    lambda: [pins.test_quantize_matches_exact_bruteforce(d, 130, 64, 5, q)
+             for d in ("f32", "bf16") for q in ("nf4", "fp4")],
+    lambda: [pins.test_division_knife_edges_match_exact_quotient(q) for q in ("nf4", "fp4")],
+    lambda: [pins.test_dequant_double_rounding_edges(q, o) for q in ("nf4", "fp4") for o in ("bf16", "f16")],
+    lambda: pins.test_f32_to_16bit_rne_against_torch_and_numpy(),
+    lambda: pins.test_matmul_one_hot_gives_weight_column(),
+    lambda: [pins.test_matmul_and_backward_exact_bruteforce(q) for q in ("nf4",)],
+]
+
+
+def _build_mutant(tmp, before, after):
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor not unique: {before!r}"
+    d = os.path.join(tmp, "m")
+    os.makedirs(d)
+    shutil.copy(os.path.join(os.path.dirname(SRC), "bnb4_oracle.h"), d)
+    with open(os.path.join(d, "bnb4_oracle.c"), "w") as f:
+        f.write(src.replace(before, after))
+    so = os.path.join(d, "libmutant.so")
+    subprocess.check_call(["cc", "-O1", "-std=c11", "-fno-fast-math", "-ffp-contract=off",
+                           "-shared", "-fPIC", "-o", so, os.path.join(d, "bnb4_oracle.c"), "-lm"])
+    return so
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    before, after = MUTATIONS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _build_mutant(tmp, before, after)
+        real = oracle.lib()
+        mutant = ctypes.CDLL(so)
+        # same signatures as the real library
+        for attr in ("oracle_code_table", "oracle_to_f32_array", "oracle_from_f32_array",
+                     "oracle_quantize", "oracle_dequantize", "oracle_matmul",
+                     "oracle_matmul_entries", "oracle_matmul_backward",
+                     "oracle_matmul_backward_entries"):
+            f, g = getattr(real, attr), getattr(mutant, attr)
+            g.restype, g.argtypes = f.restype, f.argtypes
+        monkeypatch.setattr(oracle, "_lib", mutant)
+        caught = 0
+        for check in PIN_CHECKS:
+            try:
+                check()
+            except (AssertionError, ValueError):
+                caught += 1
+        assert caught > 0, f"no pin caught mutation {name}"

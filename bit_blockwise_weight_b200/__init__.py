@@ -1,0 +1,179 @@
+"""Python binding of libbnb4.so: 4-bit blockwise weight quantization on B200.
+
+Two layers, both argument marshalling only (every step of the computation
+runs in the library's CUDA kernels):
+
+* ``bnb4_quantize``, ``bnb4_dequantize``, ``bnb4_gemv``, ``bnb4_gemm``,
+  ``bnb4_gemm_backward``: the C ABI of ``include/bnb4.h`` one to one (raw
+  device pointers as ints, sizes, enums, a ``cudaStream_t`` as an int).
+  They return the integer status.
+* ``quantize_4bit``, ``dequantize_4bit``, ``gemv_4bit``, ``gemm_4bit``,
+  ``gemm_4bit_backward``: take torch CUDA tensors, allocate outputs with
+  torch, call the C ABI on the current stream and raise ``Bnb4Error`` on a
+  non-OK status.
+
+Importing the package loads the shared library and fails loudly if it is
+missing.  There is no CPU or pure-PyTorch fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbnb4.so")
+
+NF4, FP4 = 0, 1
+F32, F16, BF16 = 0, 1, 2
+QTYPES = {"nf4": NF4, "fp4": FP4}
+STATUS_OK = 0
+
+
+class Bnb4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"libbnb4.so not found at {LIB_PATH}; build it with "
+            "`python -m bit_blockwise_weight_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    sigs = {
+        "bnb4_version": (I, []),
+        "bnb4_status_string": (ctypes.c_char_p, [I]),
+        "bnb4_quantize": (I, [P, P, P, I64, I, I, I, P]),
+        "bnb4_dequantize": (I, [P, P, P, I64, I, I, I, P]),
+        "bnb4_gemv": (I, [P, P, P, P, P, I64, I64, I, I, I, P]),
+        "bnb4_gemm": (I, [P, P, P, P, P, I64, I64, I64, I, I, I, P]),
+        "bnb4_gemm_backward": (I, [P, P, P, P, I64, I64, I64, I, I, I, P]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    return L
+
+
+_lib = _load()
+
+# ------------------------------------------------------------------ C ABI
+
+bnb4_version = _lib.bnb4_version
+bnb4_quantize = _lib.bnb4_quantize
+bnb4_dequantize = _lib.bnb4_dequantize
+bnb4_gemv = _lib.bnb4_gemv
+bnb4_gemm = _lib.bnb4_gemm
+bnb4_gemm_backward = _lib.bnb4_gemm_backward
+
+
+def status_string(status: int) -> str:
+    return _lib.bnb4_status_string(int(status)).decode()
+
+
+def library_path() -> str:
+    return LIB_PATH
+
+
+# ------------------------------------------------------- torch-level wrappers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    codes = {torch.float32: F32, torch.float16: F16, torch.bfloat16: BF16}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _qtype(q) -> int:
+    return QTYPES[q] if isinstance(q, str) else int(q)
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(status: int, what: str):
+    if status != STATUS_OK:
+        raise Bnb4Error(status, what)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def quantize_4bit(x, blocksize: int = 64, quant_type="nf4", stream=None):
+    """x: any-shape f32/f16/bf16 CUDA tensor -> (packed uint8[ceil(n/2)], absmax f32[ceil(n/B)])."""
+    torch = _torch()
+    _need_cuda(x)
+    n = x.numel()
+    packed = torch.empty((n + 1) // 2, dtype=torch.uint8, device=x.device)
+    absmax = torch.empty((n + blocksize - 1) // blocksize, dtype=torch.float32, device=x.device)
+    _check(bnb4_quantize(_ptr(x), _ptr(packed), _ptr(absmax), n, blocksize, _qtype(quant_type),
+                         _dtype_code(x), _stream(stream)), "bnb4_quantize")
+    return packed, absmax
+
+
+def dequantize_4bit(packed, absmax, n: int, blocksize: int = 64, quant_type="nf4",
+                    dtype=None, out=None, stream=None):
+    """-> out[n] of dtype (default bfloat16)."""
+    torch = _torch()
+    _need_cuda(packed, absmax)
+    if out is None:
+        out = torch.empty(n, dtype=dtype or torch.bfloat16, device=packed.device)
+    _need_cuda(out)
+    _check(bnb4_dequantize(_ptr(packed), _ptr(absmax), _ptr(out), n, blocksize,
+                           _qtype(quant_type), _dtype_code(out), _stream(stream)),
+           "bnb4_dequantize")
+    return out
+
+
+def gemv_4bit(x, packed, absmax, N: int, K: int, bias=None, blocksize: int = 64,
+              quant_type="nf4", out=None, stream=None):
+    """x [K] -> y [N] = x @ dequant(W)^T (+ bias)."""
+    torch = _torch()
+    _need_cuda(x, packed, absmax, bias)
+    y = out if out is not None else torch.empty(N, dtype=x.dtype, device=x.device)
+    _check(bnb4_gemv(_ptr(x), _ptr(packed), _ptr(absmax), _ptr(bias), _ptr(y), N, K, blocksize,
+                     _qtype(quant_type), _dtype_code(x), _stream(stream)), "bnb4_gemv")
+    return y
+
+
+def gemm_4bit(X, packed, absmax, N: int, bias=None, blocksize: int = 64, quant_type="nf4",
+              out=None, stream=None):
+    """X [M, K] -> Y [M, N] = X @ dequant(W)^T (+ bias)."""
+    torch = _torch()
+    _need_cuda(X, packed, absmax, bias)
+    M, K = X.shape
+    Y = out if out is not None else torch.empty(M, N, dtype=X.dtype, device=X.device)
+    _check(bnb4_gemm(_ptr(X), _ptr(packed), _ptr(absmax), _ptr(bias), _ptr(Y), M, N, K, blocksize,
+                     _qtype(quant_type), _dtype_code(X), _stream(stream)), "bnb4_gemm")
+    return Y
+
+
+def gemm_4bit_backward(dY, packed, absmax, K: int, blocksize: int = 64, quant_type="nf4",
+                       out=None, stream=None):
+    """dY [M, N] -> dX [M, K] = dY @ dequant(W)."""
+    torch = _torch()
+    _need_cuda(dY, packed, absmax)
+    M, N = dY.shape
+    dX = out if out is not None else torch.empty(M, K, dtype=dY.dtype, device=dY.device)
+    _check(bnb4_gemm_backward(_ptr(dY), _ptr(packed), _ptr(absmax), _ptr(dX), M, N, K, blocksize,
+                              _qtype(quant_type), _dtype_code(dY), _stream(stream)),
+           "bnb4_gemm_backward")
+    return dX

@@ -1,0 +1,133 @@
+// api.cu -- the C ABI of libbnb4.so (declared in include/bnb4.h).
+//
+// Each entry point validates its arguments on the host, picks a kernel and
+// enqueues it on the caller's stream.  Nothing is allocated, nothing is
+// synchronised, and a failed check enqueues nothing.  There is no fallback:
+// an input the kernels do not handle is an error.
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bnb4 {
+
+int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+            v = 148;
+        cache[dev].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_blocksize(int b) {
+    return b >= 64 && b <= 4096 && (b & (b - 1)) == 0;
+}
+
+bool valid_qtype(bnb4_quant_type q) { return q == BNB4_NF4 || q == BNB4_FP4; }
+
+bool valid_dtype(bnb4_dtype d) { return d == BNB4_F32 || d == BNB4_F16 || d == BNB4_BF16; }
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+
+bnb4_status check_matmul(const void *a, const uint8_t *W, const float *absmax, const void *bias,
+                         const void *out, int64_t M, int64_t N, int64_t K, int blocksize,
+                         bnb4_quant_type qt, bnb4_dtype dt) {
+    if (!a || !W || !absmax || !out) return BNB4_ERR_NULL;
+    if (!aligned16(a) || !aligned16(W) || !aligned16(absmax) || !aligned16(out) ||
+        (bias && !aligned16(bias)))
+        return BNB4_ERR_ALIGN;
+    if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
+    if (!valid_qtype(qt)) return BNB4_ERR_QTYPE;
+    if (dt != BNB4_F16 && dt != BNB4_BF16) return BNB4_ERR_DTYPE;
+    if (M < 1 || N < 1 || K < 1 || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim)
+        return BNB4_ERR_SHAPE;
+    if (K % 32 != 0 || K % blocksize != 0) return BNB4_ERR_SHAPE;
+    return BNB4_OK;
+}
+
+bnb4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA; }
+
+}  // namespace
+}  // namespace bnb4
+
+using namespace bnb4;
+
+extern "C" {
+
+int bnb4_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char *bnb4_status_string(bnb4_status s) {
+    switch (s) {
+    case BNB4_OK: return "ok";
+    case BNB4_ERR_NULL: return "a required pointer is NULL";
+    case BNB4_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case BNB4_ERR_BLOCKSIZE: return "blocksize must be a power of two in [64, 4096]";
+    case BNB4_ERR_SHAPE: return "invalid shape (sizes, K % blocksize, K % 32)";
+    case BNB4_ERR_DTYPE: return "dtype not supported by this call";
+    case BNB4_ERR_QTYPE: return "quant type must be NF4 or FP4";
+    case BNB4_ERR_CUDA: return "CUDA kernel launch failed";
+    case BNB4_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+bnb4_status bnb4_quantize(const void *x, uint8_t *packed, float *absmax, int64_t n, int blocksize,
+                          bnb4_quant_type qt, bnb4_dtype dt, cudaStream_t stream) {
+    if (n < 0) return BNB4_ERR_SHAPE;
+    if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
+    if (!valid_qtype(qt)) return BNB4_ERR_QTYPE;
+    if (!valid_dtype(dt)) return BNB4_ERR_DTYPE;
+    if (n == 0) return BNB4_OK;
+    if (!x || !packed || !absmax) return BNB4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(absmax)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_quantize(x, packed, absmax, n, blocksize, qt, dt, stream));
+}
+
+bnb4_status bnb4_dequantize(const uint8_t *packed, const float *absmax, void *out, int64_t n,
+                            int blocksize, bnb4_quant_type qt, bnb4_dtype dt, cudaStream_t stream) {
+    if (n < 0) return BNB4_ERR_SHAPE;
+    if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
+    if (!valid_qtype(qt)) return BNB4_ERR_QTYPE;
+    if (!valid_dtype(dt)) return BNB4_ERR_DTYPE;
+    if (n == 0) return BNB4_OK;
+    if (!packed || !absmax || !out) return BNB4_ERR_NULL;
+    if (!aligned16(packed) || !aligned16(absmax) || !aligned16(out)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_dequantize(packed, absmax, out, n, blocksize, qt, dt, stream));
+}
+
+bnb4_status bnb4_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
+                      void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
+                      bnb4_dtype dt, cudaStream_t stream) {
+    bnb4_status s = check_matmul(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt);
+    if (s != BNB4_OK) return s;
+    return from_cuda(launch_gemv(x, W, absmax, bias, y, N, K, blocksize, qt, dt, stream));
+}
+
+bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, const void *bias,
+                      void *Y, int64_t M, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
+                      bnb4_dtype dt, cudaStream_t stream) {
+    bnb4_status s = check_matmul(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt);
+    if (s != BNB4_OK) return s;
+    if (M <= kSmallMMax)
+        return from_cuda(launch_gemm_small(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, stream));
+    return from_cuda(launch_gemm_tc(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, false, stream));
+}
+
+bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *absmax, void *dX,
+                               int64_t M, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
+                               bnb4_dtype dt, cudaStream_t stream) {
+    bnb4_status s = check_matmul(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt);
+    if (s != BNB4_OK) return s;
+    return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true, stream));
+}
+
+}  // extern "C"

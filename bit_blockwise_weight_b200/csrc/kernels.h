@@ -1,0 +1,44 @@
+// kernels.h -- host launchers for the libbnb4 kernels (internal to the library).
+// Arguments have been validated by the C ABI layer (api.cu) before these run.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bnb4.h"
+
+namespace bnb4 {
+
+// number of SMs of the current device (cached per device)
+int device_sm_count();
+
+cudaError_t launch_quantize(const void *x, uint8_t *packed, float *absmax, int64_t n,
+                            int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+                            cudaStream_t stream);
+
+cudaError_t launch_dequantize(const uint8_t *packed, const float *absmax, void *out, int64_t n,
+                              int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+                              cudaStream_t stream);
+
+// M == 1, CUDA cores
+cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
+                        void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
+                        bnb4_dtype dt, cudaStream_t stream);
+
+// 1 <= M <= 16: weights decoded in registers into mma.sync fragments
+cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
+                              const void *bias, void *Y, int64_t M, int64_t N, int64_t K,
+                              int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+                              cudaStream_t stream);
+
+// large M: tcgen05 with weight tiles dequantized into shared memory.
+// backward == true computes dX[M, K] = dY[M, N] @ dequant(W) instead.
+cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax,
+                           const void *bias, void *D, int64_t M, int64_t N, int64_t K,
+                           int blocksize, bnb4_quant_type qt, bnb4_dtype dt, bool backward,
+                           cudaStream_t stream);
+
+// largest M handled by launch_gemm_small
+constexpr int64_t kSmallMMax = 16;
+
+}  // namespace bnb4

@@ -1,0 +1,87 @@
+// tables.cu -- host construction of the code tables and of the decision
+// tables that the quantize kernel searches (see common.cuh).
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+
+#include "common.cuh"
+
+namespace bnb4 {
+
+CodeTable host_code_table(bnb4_quant_type qt) {
+    CodeTable t{};
+    if (qt == BNB4_NF4) {
+        static const float nf4[16] = {
+            -1.0f,       -0.6961928f, -0.5250731f, -0.3949175f, -0.2844414f, -0.1848074f,
+            -0.0910500f, 0.0f,        0.0795803f,  0.1609302f,  0.2461123f,  0.3379152f,
+            0.4407098f,  0.5626170f,  0.7229568f,  1.0f};
+        for (int i = 0; i < 16; ++i) t.v[i] = nf4[i];
+    } else {
+        // E2M1 -> value / 6
+        for (int i = 0; i < 16; ++i) {
+            const int sign = i >> 3, e = (i >> 1) & 3, m = i & 1;
+            const double mag = e ? std::ldexp(2.0 + m, e - 2) : 0.5 * m;
+            t.v[i] = (float)((sign ? -mag : mag) / 6.0);
+        }
+    }
+    return t;
+}
+
+// cell index of an fp32 value, exactly as the device computes it:
+// rn(13 v + 13) with ties to even (13 v + 13 is exact in double).
+static int host_cell(float v) { return (int)std::nearbyint(13.0 * (double)v + 13.0); }
+
+QuantTables host_quant_tables(bnb4_quant_type qt) {
+    const CodeTable c = host_code_table(qt);
+    // distinct values in ascending order, each with the smallest index holding it
+    float val[16];
+    int idx[16];
+    int nd = 0;
+    for (int i = 0; i < 16; ++i) {
+        bool seen = false;
+        for (int j = 0; j < nd; ++j)
+            if (val[j] == c.v[i]) seen = true;  // +0 == -0: keeps index 0
+        if (!seen) {
+            val[nd] = c.v[i];
+            idx[nd] = i;
+            ++nd;
+        }
+    }
+    for (int a = 1; a < nd; ++a)  // insertion sort by value
+        for (int b = a; b > 0 && val[b - 1] > val[b]; --b) {
+            float tv = val[b]; val[b] = val[b - 1]; val[b - 1] = tv;
+            int ti = idx[b]; idx[b] = idx[b - 1]; idx[b - 1] = ti;
+        }
+    // thresholds: v > thr[r]  <=>  rank(v) >= r + 1
+    float thr[16];
+    for (int r = 0; r + 1 < nd; ++r) {
+        const double mid = 0.5 * ((double)val[r] + (double)val[r + 1]);  // exact
+        const bool tie_up = idx[r + 1] < idx[r];  // a tie goes to the smaller index
+        float t = (float)mid;
+        if ((double)t > mid) t = std::nextafter(t, -INFINITY);
+        if (tie_up && (double)t == mid) t = std::nextafter(t, -INFINITY);
+        thr[r] = t;
+    }
+    QuantTables q{};
+    for (int k = 0; k < 32; ++k) {
+        int base = 0, inside = -1;
+        for (int r = 0; r + 1 < nd; ++r) {
+            const int cr = host_cell(thr[r]);
+            if (cr < k) ++base;
+            if (cr == k) {
+                if (inside >= 0) {
+                    std::fprintf(stderr, "bnb4: two thresholds in one cell\n");
+                    std::abort();
+                }
+                inside = r;
+            }
+        }
+        const int lo = idx[base];
+        const int hi = inside >= 0 ? idx[base + 1] : lo;
+        q.thr[k] = inside >= 0 ? thr[inside] : 2.0f;  // 2 > every |v| <= 1
+        q.lohi[k] = (uint32_t)lo | ((uint32_t)hi << 4);
+    }
+    return q;
+}
+
+}  // namespace bnb4

@@ -1,0 +1,155 @@
+/*
+ * bnb4.h -- C ABI of libbnb4.so: 4-bit blockwise weight quantization (NF4 /
+ * FP4) and the 4-bit matmuls that consume it, on NVIDIA B200 (sm_100a).
+ *
+ * Operations and where they are defined (page title, section):
+ *   bnb4_quantize       "mps-bitsandbytes 0.4.7", Functional API
+ *                       (quantize_nf4 / quantize_fp4 -> (packed, absmax)),
+ *                       Features table (NF4, FP4); "Feat/mps gemm 4bit bf16",
+ *                       What runs natively now (quantize_4bit).
+ *   bnb4_dequantize     same pages (dequantize_nf4, dequantize_4bit and its
+ *                       .out form: the caller gives the output buffer).
+ *   bnb4_gemv           "Feat/mps gemm 4bit bf16", What runs natively now
+ *                       (gemv_4bit, M == 1, fused dequant + dot) and
+ *                       Correctness (bias epilogue); "mps-bitsandbytes
+ *                       0.4.7", Functional API (matmul_nf4(..., bias=None)).
+ *   bnb4_gemm           "Feat/mps gemm 4bit bf16", What runs natively now
+ *                       (gemm_4bit, general M).
+ *   bnb4_gemm_backward  "Feat/mps gemm 4bit bf16", What runs natively now and
+ *                       the paragraph on the new op: grad_input =
+ *                       grad_output @ dequantize_4bit(B).
+ *
+ * Numeric contract (the readings of the pages that the CPU oracle follows):
+ *   - absmax[b] = max |x_i| over block b, in fp32; blocks are `blocksize`
+ *     consecutive elements of the flat input; the last block may be short.
+ *   - v = x / absmax[b] as an IEEE fp32 quotient (v = 0 when absmax == 0).
+ *   - code index = argmin_i |v - code[i]| over the 16-entry table, ties to the
+ *     smallest index.  NF4 table: the 16 values listed with the gemv NF4
+ *     workload; FP4 table: E2M1 (index = sign<<3 | exp<<1 | mant, bias 1,
+ *     subnormals) divided by 6 so that the largest magnitude is 1.
+ *   - packing: byte j = idx[2j] << 4 | idx[2j+1] (first element in the high
+ *     nibble); an odd last element leaves the low nibble 0.
+ *   - dequantized value = RN_dtype(fp32(code[idx] * absmax)): one fp32
+ *     product, then one round-to-nearest-even conversion.
+ *   - matmuls accumulate in fp32.  They consume the weight dequantized as
+ *     above and rounded to the compute dtype (bf16 / fp16); the result is
+ *     rounded once to the compute dtype.  The bias, if given, is added in
+ *     fp32 before that rounding.
+ *
+ * Weight layout for the matmuls: W is [N, K] row-major (out x in, like a
+ * Linear layer's weight) and was quantized as one flat array of N*K
+ * elements, so that with K % blocksize == 0 every block lies in one row:
+ *   packedW  uint8 [N, K/2]           absmax  float32 [N, K/blocksize].
+ *
+ * Ownership and execution:
+ *   - Every pointer is a device pointer owned by the caller.  The library
+ *     allocates no memory and holds no per-call state.
+ *   - Every call is asynchronous on `stream` (0 = the legacy default stream)
+ *     and never synchronises the host.  Inputs must stay valid, and outputs
+ *     must not be read, until work enqueued on `stream` has completed.
+ *   - Calls on different streams may run concurrently on disjoint outputs.
+ *
+ * Errors: each call returns a bnb4_status.  Argument checks happen on the
+ * host before anything is enqueued; on any error nothing is enqueued and no
+ * output is touched.  BNB4_ERR_CUDA reports a launch failure (the CUDA error
+ * is left for the caller's next cudaGetLastError / synchronisation).  No call
+ * ever falls back to another implementation.
+ */
+#ifndef BNB4_H
+#define BNB4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#ifndef __CUDA_RUNTIME_H__
+/* Same underlying type as cuda_runtime_api.h's cudaStream_t. */
+typedef struct CUstream_st *cudaStream_t;
+#endif
+
+typedef enum { BNB4_NF4 = 0, BNB4_FP4 = 1 } bnb4_quant_type;
+
+typedef enum { BNB4_F32 = 0, BNB4_F16 = 1, BNB4_BF16 = 2 } bnb4_dtype;
+
+typedef enum {
+    BNB4_OK = 0,
+    BNB4_ERR_NULL = 1,      /* a required pointer is NULL                     */
+    BNB4_ERR_ALIGN = 2,     /* a pointer is not 16-byte aligned               */
+    BNB4_ERR_BLOCKSIZE = 3, /* blocksize not in {64,128,...,4096}             */
+    BNB4_ERR_SHAPE = 4,     /* negative size, K % blocksize, K % 32, too big  */
+    BNB4_ERR_DTYPE = 5,     /* dtype not accepted by this call                */
+    BNB4_ERR_QTYPE = 6,     /* quant type not NF4 / FP4                       */
+    BNB4_ERR_CUDA = 7,      /* a kernel launch failed                         */
+    BNB4_ERR_TIMEOUT = 8    /* a bounded device-side wait gave up             */
+} bnb4_status;
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int bnb4_version(void);
+
+/* Static text for a status code (never NULL). */
+const char *bnb4_status_string(bnb4_status status);
+
+/*
+ * Quantize n elements of x.
+ *   x        [n] of x_dtype (f32 / f16 / bf16), 16-byte aligned.
+ *   packed   [ceil(n/2)] bytes out, 16-byte aligned.
+ *   absmax   [ceil(n/blocksize)] float32 out, 16-byte aligned.
+ *   n >= 0 (n == 0 enqueues nothing); blocksize in {64, 128, ..., 4096}.
+ */
+bnb4_status bnb4_quantize(const void *x, uint8_t *packed, float *absmax,
+                          int64_t n, int blocksize, bnb4_quant_type quant_type,
+                          bnb4_dtype x_dtype, cudaStream_t stream);
+
+/*
+ * Dequantize n elements: out[i] = RN_out_dtype(fp32(code[idx_i] * absmax[i / blocksize])).
+ *   packed   [ceil(n/2)] bytes, absmax [ceil(n/blocksize)] float32,
+ *   out      [n] of out_dtype (f32 / f16 / bf16); all 16-byte aligned.
+ */
+bnb4_status bnb4_dequantize(const uint8_t *packed, const float *absmax,
+                            void *out, int64_t n, int blocksize,
+                            bnb4_quant_type quant_type, bnb4_dtype out_dtype,
+                            cudaStream_t stream);
+
+/*
+ * Matrix-vector product for decode (M == 1): y = x @ dequant(W)^T (+ bias).
+ *   x        [K] of dt;  packedW [N, K/2];  absmax [N, K/blocksize];
+ *   bias     [N] of dt or NULL;  y [N] of dt (out).
+ *   dt in {f16, bf16}; K % blocksize == 0 and K % 32 == 0; N, K >= 1.
+ */
+bnb4_status bnb4_gemv(const void *x, const uint8_t *packedW,
+                      const float *absmax, const void *bias, void *y,
+                      int64_t N, int64_t K, int blocksize,
+                      bnb4_quant_type quant_type, bnb4_dtype dt,
+                      cudaStream_t stream);
+
+/*
+ * General matmul: Y[M, N] = X[M, K] @ dequant(W)^T (+ bias), row-major.
+ *   X [M, K] of dt;  bias [N] of dt or NULL;  Y [M, N] of dt (out).
+ *   Same constraints as bnb4_gemv; M >= 1.  Small M streams the weight once
+ *   through a register-decode tensor-core kernel, large M runs the tcgen05
+ *   kernel that dequantizes weight tiles into shared memory.
+ */
+bnb4_status bnb4_gemm(const void *X, const uint8_t *packedW,
+                      const float *absmax, const void *bias, void *Y,
+                      int64_t M, int64_t N, int64_t K, int blocksize,
+                      bnb4_quant_type quant_type, bnb4_dtype dt,
+                      cudaStream_t stream);
+
+/*
+ * Backward of bnb4_gemm with respect to its input:
+ *   dX[M, K] = dY[M, N] @ dequant(W)   (reduction over N, no bias term).
+ *   dY [M, N] of dt;  dX [M, K] of dt (out); same weight arguments and
+ *   constraints as bnb4_gemm.
+ */
+bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *packedW,
+                               const float *absmax, void *dX, int64_t M,
+                               int64_t N, int64_t K, int blocksize,
+                               bnb4_quant_type quant_type, bnb4_dtype dt,
+                               cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BNB4_H */

@@ -1,0 +1,105 @@
+"""gemv_4bit / gemm_4bit / gemm_4bit_backward on the GPU against the float64 oracle.
+
+Bar: relative L2 error <= 5e-3 (bf16/fp16 out, fp32 accumulate) against the
+float64 product of the oracle's dequantized (fp32) weights.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_blockwise_weight_b200 as bnb4
+import oracle
+from bit_blockwise_weight_b200 import synthetic
+
+from gpu_util import MATMUL_TOL, as_f64, rel_l2, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+class Weight:
+    """A seeded fp32 weight [N, K] quantized by the oracle (the GPU path gets the same bytes)."""
+
+    def __init__(self, N, K, B=64, q="nf4", seed=0, sigma=0.02):
+        self.N, self.K, self.B, self.q = N, K, B, q
+        w = synthetic.weight(N, K, seed, sigma).numpy().reshape(-1)
+        self.packed, self.absmax = oracle.quantize(w, "f32", B, q)
+        self.dp = torch.from_numpy(self.packed).cuda()
+        self.da = torch.from_numpy(self.absmax).cuda()
+
+
+def _ref_forward(Wt, Xs, dt, bias_s, rows=None):
+    M = Xs.size // Wt.K
+    if rows is None:
+        return oracle.matmul(Xs, dt, Wt.packed, Wt.absmax, bias_s, M, Wt.N, Wt.K, Wt.B, Wt.q)
+    ms = np.repeat(np.arange(M), rows.size)
+    js = np.tile(rows, M)
+    v = oracle.matmul_entries(Xs, dt, Wt.packed, Wt.absmax, bias_s, M, Wt.N, Wt.K, Wt.B, Wt.q,
+                              ms, js)
+    return v.reshape(M, rows.size)
+
+
+# ----------------------------------------------------------------------- gemv
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("N,K,B", [(96, 4096, 64), (33, 512, 128), (70, 4672, 64),
+                                   (64, 2048, 2048), (200, 1024, 1024), (17, 128, 64),
+                                   (40, 8192, 4096)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemv_small_shapes(q, dt, N, K, B, with_bias):
+    Wt = Weight(N, K, B, q, seed=N + K)
+    xs = synthetic.storage_numpy(synthetic.activations(1, K, seed=1, dtype=dt)).reshape(-1)
+    bs = synthetic.storage_numpy(synthetic.bias(N, seed=2, dtype=dt)) if with_bias else None
+    y = bnb4.gemv_4bit(to_dev(xs, dt), Wt.dp, Wt.da, N, K, None if bs is None else to_dev(bs, dt),
+                       B, q)
+    ref = _ref_forward(Wt, xs, dt, bs)[0]
+    err = rel_l2(as_f64(to_host(y), dt), ref)
+    assert err <= MATMUL_TOL, err
+
+
+@pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_gemv_llama_decode_shapes_sampled(K, N, with_bias):
+    """Llama-3-8B-shaped decode projections, NF4 blocksize 64, bf16: sampled rows."""
+    Wt = Weight(N, K, 64, "nf4", seed=0, sigma=0.02)
+    xs = synthetic.storage_numpy(synthetic.activations(1, K, seed=1)).reshape(-1)
+    bs = synthetic.storage_numpy(synthetic.bias(N, seed=2)) if with_bias else None
+    y = to_host(bnb4.gemv_4bit(to_dev(xs, "bf16"), Wt.dp, Wt.da, N, K,
+                               None if bs is None else to_dev(bs, "bf16"), 64, "nf4"))
+    rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(K + N).integers(0, N, 254)]))
+    ref = _ref_forward(Wt, xs, "bf16", bs, rows)[0]
+    err = rel_l2(as_f64(y, "bf16")[rows], ref)
+    assert err <= MATMUL_TOL, err
+
+
+# -------------------------------------------------------------- small-M gemm
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 8, 9, 16])
+@pytest.mark.parametrize("N,K,B", [(96, 2048, 64), (45, 1600, 64), (64, 4096, 256),
+                                   (33, 1024, 1024)])
+def test_gemm_small_m(q, dt, M, N, K, B):
+    Wt = Weight(N, K, B, q, seed=M + N)
+    Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
+    bs = synthetic.storage_numpy(synthetic.bias(N, seed=2, dtype=dt)) if M % 2 else None
+    Y = bnb4.gemm_4bit(to_dev(Xs, dt).view(M, K), Wt.dp, Wt.da, N,
+                       None if bs is None else to_dev(bs, dt), B, q)
+    ref = _ref_forward(Wt, Xs, dt, bs)
+    err = rel_l2(as_f64(to_host(Y), dt).reshape(M, N), ref)
+    assert err <= MATMUL_TOL, err
+
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
+def test_gemm_small_m_70b_shapes_sampled(q, dt, K, N):
+    """70B-shaped projections, M in {1,2,4,8,16}, sigma 0.015: sampled rows."""
+    Wt = Weight(N, K, 64, q, seed=0, sigma=0.015)
+    rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(K).integers(0, N, 62)]))
+    for M in (1, 2, 4, 8, 16):
+        Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
+        Y = to_host(bnb4.gemm_4bit(to_dev(Xs, dt).view(M, K), Wt.dp, Wt.da, N, None, 64, q))
+        ref = _ref_forward(Wt, Xs, dt, None, rows)
+        err = rel_l2(as_f64(Y, dt).reshape(M, N)[:, rows], ref)
+        assert err <= MATMUL_TOL, (M, err)

@@ -1,0 +1,493 @@
+"""Benchmark of the 4-bit blockwise weight path on B200.
+
+One step = one pass of the whole hot path over one batch of seeded synthetic
+input:
+  1. quantize_4bit     x[2^28] bf16 ~N(0,1) + 1% x20 outliers -> NF4, blocksize 64
+  2. gemv_4bit + bias  Llama-3-8B decode projections (K,N) = (4096,4096),
+                       (4096,1024), (4096,14336), (14336,4096); NF4 B=64, bf16
+  3. gemm_4bit M=16    70B-shaped (K,N) = (8192,28672), (28672,8192)
+  4. gemm_4bit M=512   prefill, K=4096, N=14336
+  5. gemm_4bit_backward M=512 (grad_input = grad_out @ dequant(W))
+  6. dequantize_4bit   the step-1 result back to bf16 (after 2-5 have evicted it from L2)
+Throughput (GB/s) = algorithmic bytes of the step / step time; the step's
+working set (~1.6 GB) is far larger than L2, so every kernel reads cold data.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (the plain C restatement of the
+method) on a bounded sample of the same workload.  Under torchrun every rank
+runs its own independent batch (weak scaling, no collective on the data
+path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+N_ELEMS = 1 << 28
+BLOCK = 64
+GEMV_SHAPES = [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)]
+SMALLM_SHAPES = [(8192, 28672), (28672, 8192)]
+SMALLM_M = 16
+PREFILL = (512, 4096, 14336)  # M, K, N
+METRIC = "gemv_4bit NF4 decode GB/s & % of HBM roofline; quantize_4bit GB/s"
+WORKLOAD = ("full 4-bit hot path per step: quantize 2^28 bf16 (NF4, B=64) + gemv+bias on 4 "
+            "Llama-3-8B decode shapes + M=16 gemm on 2 70B shapes + M=512 prefill gemm "
+            "(K=4096, N=14336) and its backward + dequantize 2^28")
+
+
+def wbytes(N, K):
+    return N * K // 2 + N * K // BLOCK * 4
+
+
+def step_ops():
+    """(name, algorithmic bytes, flops) for each launch of one step, in order."""
+    ops = [("quantize_4bit", N_ELEMS * 2 + N_ELEMS // 2 + N_ELEMS // BLOCK * 4, 0)]
+    for K, N in GEMV_SHAPES:
+        ops.append((f"gemv_4bit_{K}x{N}", wbytes(N, K) + 2 * K + 2 * N + 2 * N, 2 * N * K))
+    for K, N in SMALLM_SHAPES:
+        M = SMALLM_M
+        ops.append((f"gemm_4bit_M{M}_{K}x{N}", wbytes(N, K) + 2 * M * K + 2 * M * N, 2 * M * N * K))
+    M, K, N = PREFILL
+    ops.append((f"gemm_4bit_M{M}_{K}x{N}", wbytes(N, K) + 2 * M * K + 2 * M * N, 2 * M * N * K))
+    ops.append((f"gemm_4bit_backward_M{M}_{K}x{N}", wbytes(N, K) + 2 * M * N + 2 * M * K,
+                2 * M * N * K))
+    ops.append(("dequantize_4bit", N_ELEMS // 2 + N_ELEMS // BLOCK * 4 + N_ELEMS * 2, 0))
+    return ops
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained", p["bf16_tflops"]), \
+            "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_src_hash(fname):
+    with open(os.path.join(ROOT, "bit_blockwise_weight_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(op_name):
+    """DRAM bytes per launch recorded by an ncu capture under profiles/, or None when
+    the kernel source has changed since (the summary records the source hash)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(op_name)
+    except (OSError, ValueError):
+        return None
+    if not rec or rec.get("src_sha256_16") != kernel_src_hash(rec["src"]):
+        return None
+    return rec["dram_bytes_per_launch"]
+
+
+SRC_OF = {"quantize_4bit": "quant.cu", "dequantize_4bit": "quant.cu"}
+
+
+def src_of(op):
+    if op in SRC_OF:
+        return SRC_OF[op]
+    if op.startswith("gemv"):
+        return "gemv.cu"
+    if "backward" in op or "_M512_" in op:
+        return "gemm_tc.cu"
+    return "gemm_small.cu"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.rows = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([c.strip() for c in line.split(",")])
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm = [float(r[1]) for r in self.rows if len(r) >= 9 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if len(r) >= 9 and r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            if len(r) < 9:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- our arm
+
+class Step:
+    """Device buffers for one batch and the launch sequence of one step."""
+
+    def __init__(self, dev, seed):
+        import bit_blockwise_weight_b200 as bnb4
+        from bit_blockwise_weight_b200 import synthetic
+        self.bnb4 = bnb4
+        d = str(dev)
+        self.x = synthetic.roundtrip_tensor(N_ELEMS, seed, "bf16", device=d)
+        self.packed = torch.empty(N_ELEMS // 2, dtype=torch.uint8, device=dev)
+        self.absmax = torch.empty(N_ELEMS // BLOCK, dtype=torch.float32, device=dev)
+        self.deq = torch.empty(N_ELEMS, dtype=torch.bfloat16, device=dev)
+
+        def qweight(N, K, sigma, s):
+            w = synthetic.normal((N * K,), s, sigma, "f32", device=d)
+            p, a = bnb4.quantize_4bit(w, BLOCK, "nf4")
+            del w
+            return p, a
+
+        self.gemv = []
+        for i, (K, N) in enumerate(GEMV_SHAPES):
+            p, a = qweight(N, K, 0.02, 100 * seed + i)
+            xv = synthetic.normal((K,), 1000 + seed, 1.0, "bf16", device=d)
+            b = synthetic.normal((N,), 2000 + seed, 1.0, "bf16", device=d)
+            self.gemv.append((K, N, p, a, xv, b, torch.empty(N, dtype=torch.bfloat16, device=dev)))
+        self.smallm = []
+        for i, (K, N) in enumerate(SMALLM_SHAPES):
+            p, a = qweight(N, K, 0.015, 100 * seed + 10 + i)
+            X = synthetic.normal((SMALLM_M, K), 3000 + seed + i, 1.0, "bf16", device=d)
+            self.smallm.append((K, N, p, a, X,
+                                torch.empty(SMALLM_M, N, dtype=torch.bfloat16, device=dev)))
+        M, K, N = PREFILL
+        p, a = qweight(N, K, 0.02, 100 * seed + 20)
+        X = synthetic.normal((M, K), 4000 + seed, 1.0, "bf16", device=d)
+        dY = synthetic.normal((M, N), 5000 + seed, 1.0, "bf16", device=d)
+        self.prefill = (M, K, N, p, a, X, dY, torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                        torch.empty(M, K, dtype=torch.bfloat16, device=dev))
+        torch.cuda.synchronize(dev)
+
+    def launches(self):
+        """The step as a list of zero-argument callables, one per kernel launch."""
+        b = self.bnb4
+        L = [lambda: b.quantize_4bit_into(self.x, self.packed, self.absmax, BLOCK, "nf4")]
+        for K, N, p, a, xv, bias, y in self.gemv:
+            L.append(lambda K=K, N=N, p=p, a=a, xv=xv, bias=bias, y=y:
+                     b.gemv_4bit(xv, p, a, N, K, bias, BLOCK, "nf4", out=y))
+        for K, N, p, a, X, Y in self.smallm:
+            L.append(lambda N=N, p=p, a=a, X=X, Y=Y: b.gemm_4bit(X, p, a, N, None, BLOCK, "nf4", out=Y))
+        M, K, N, p, a, X, dY, Y, dX = self.prefill
+        L.append(lambda: b.gemm_4bit(X, p, a, N, None, BLOCK, "nf4", out=Y))
+        L.append(lambda: b.gemm_4bit_backward(dY, p, a, K, BLOCK, "nf4", out=dX))
+        L.append(lambda: b.dequantize_4bit(self.packed, self.absmax, N_ELEMS, BLOCK, "nf4", out=self.deq))
+        return L
+
+
+def run_ours(args, rank, world, dev):
+    import bit_blockwise_weight_b200 as bnb4
+    hbm, tc_burst, tc_sust, peak_kind = load_peaks()
+    ops = step_ops()
+    step = Step(dev, seed=rank)
+    calls = step.launches()
+    assert len(calls) == len(ops)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        for c in calls:
+            c()
+    torch.cuda.synchronize(dev)
+
+    # per-launch events on the launching stream, inside the timed region
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if rank == 0 else -1) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    t0.record(stream)
+    for k in range(args.steps):
+        ev[k][0].record(stream)
+        for i, c in enumerate(calls):
+            c()
+            ev[k][i + 1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop() if sampler else None
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+        torch.distributed.barrier()
+
+    per_op_ms = [statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps))
+                 for i in range(len(calls))]
+    step_bytes = sum(b for _, b, _ in ops)
+    value = step_bytes * args.steps * world / (ms / 1e3) / 1e9
+
+    # e2e: the same step through the public API from pinned host buffers; the step's
+    # inputs go host->device and every output comes back device->host, every step
+    e2e = run_e2e(args, step, dev, stream)
+
+    if rank != 0:
+        return None
+    # dominant kernel by time share
+    shares = sorted(((t, i) for i, t in enumerate(per_op_ms)), reverse=True)
+    _, di = shares[0]
+    name, nbytes, nflops = ops[di]
+    if nflops and "_M512_" in name:
+        achieved = nflops / (per_op_ms[di] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_sust,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_sust, 4),
+                "traffic": profiled_traffic(name), "kernel": name,
+                "peak_kind": f"{peak_kind} sustained bf16"}
+    else:
+        achieved = nbytes / (per_op_ms[di] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(name),
+                "kernel": name, "peak_kind": f"{peak_kind} HBM copy"}
+    parts = {}
+    for (nm, nb, nf), t in zip(ops, per_op_ms):
+        e = {"us": round(t * 1e3, 2), "GB/s": round(nb / (t / 1e3) / 1e9, 1),
+             "hbm_frac": round(nb / (t / 1e3) / 1e9 / hbm, 4),
+             "share": round(t / sum(per_op_ms), 4)}
+        if "_M512_" in nm:
+            e["TFLOP/s"] = round(nf / (t / 1e3) / 1e12, 1)
+            e["tensor_frac"] = round(nf / (t / 1e3) / 1e12 / tc_sust, 4)
+        parts[nm] = e
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) / N(0,0.02) tensors; no checkpoints)",
+        "config": {"workload": WORKLOAD, "n_elems": N_ELEMS, "quant_type": "nf4",
+                   "blocksize": BLOCK, "gemv_shapes_KN": GEMV_SHAPES,
+                   "smallm": {"M": SMALLM_M, "shapes_KN": SMALLM_SHAPES},
+                   "prefill_MKN": PREFILL, "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs larger than L2 (step working set ~1.6 GB vs 126 MB L2)"},
+        "roofline": roof,
+        "parts": parts,
+        "e2e": e2e,
+        "gpu_launches": len(calls) * args.steps,
+        "clocks": clocks,
+        "library": bnb4.library_path(),
+    }
+    if args.cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return line
+
+
+def run_e2e(args, step, dev, stream):
+    """Same step, host buffers in and out through the public API (pinned memory)."""
+    import bit_blockwise_weight_b200 as bnb4
+    h_x = step.x.cpu().pin_memory()
+    h_gemv_x = [g[4].cpu().pin_memory() for g in step.gemv]
+    h_sm_X = [s[4].cpu().pin_memory() for s in step.smallm]
+    M, K, N, p, a, X, dY, Y, dX = step.prefill
+    h_X, h_dY = X.cpu().pin_memory(), dY.cpu().pin_memory()
+    outs = [step.packed, step.absmax, step.deq] + [g[6] for g in step.gemv] + \
+        [s[5] for s in step.smallm] + [Y, dX]
+    h_outs = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    ins = [(h_x, step.x)] + [(h, g[4]) for h, g in zip(h_gemv_x, step.gemv)] + \
+        [(h, s[4]) for h, s in zip(h_sm_X, step.smallm)] + [(h_X, X), (h_dY, dY)]
+    h2d = sum(h.numel() * h.element_size() for h, _ in ins)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+    calls = step.launches()
+    steps = max(1, min(args.steps, 5))
+
+    def one():
+        for h, d in ins:
+            d.copy_(h, non_blocking=True)
+        for c in calls:
+            c()
+        for h, o in zip(h_outs, outs):
+            h.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    step_bytes = sum(b for _, b, _ in step_ops())
+    return {"value": round(step_bytes * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": round(ms / steps, 3)}
+
+
+# ------------------------------------------------------------ CPU oracle arm
+
+def oracle_sample(seconds_budget: float):
+    """Time the CPU oracle on a bounded sample of every op of the step.
+
+    Returns (extrapolated GB/s for the whole step, description, per-op detail).
+    Each op runs on a slice of its workload (a number of elements, rows or
+    output entries); its time is scaled to the full op by that fraction.
+    """
+    import numpy as np
+    import oracle
+    from bit_blockwise_weight_b200 import synthetic
+    oracle.lib()
+    ops = step_ops()
+    detail = {}
+    full_time = 0.0
+    frac_q = 1 << 24
+    x = synthetic.storage_numpy(synthetic.roundtrip_tensor(frac_q, 0, "bf16"))
+    t = time.perf_counter()
+    p, a = oracle.quantize(x, "bf16", BLOCK, "nf4")
+    tq = (time.perf_counter() - t) * (N_ELEMS / frac_q)
+    t = time.perf_counter()
+    oracle.dequantize(p, a, frac_q, BLOCK, "nf4", "bf16")
+    td = (time.perf_counter() - t) * (N_ELEMS / frac_q)
+    detail["quantize_4bit"] = f"{frac_q} elements"
+    detail["dequantize_4bit"] = f"{frac_q} elements"
+    full_time += tq + td
+
+    def mm_rows(K, N, M, rows, backward=False):
+        w = synthetic.weight(min(N, 64), K, 0).numpy().reshape(-1)
+        wp, wa = oracle.quantize(w, "f32", BLOCK, "nf4")
+        Nw = min(N, 64)
+        if backward:
+            dY = synthetic.storage_numpy(synthetic.grad_output(1, Nw, 3)).reshape(-1)
+            ks = np.arange(rows) % K
+            t = time.perf_counter()
+            oracle.matmul_backward_entries(dY, "bf16", wp, wa, 1, Nw, K, BLOCK, "nf4",
+                                           np.zeros(rows, np.int64), ks)
+            el = time.perf_counter() - t
+            return el / rows * (N / Nw) * (M * K)   # each entry sums over N
+        X = synthetic.storage_numpy(synthetic.activations(1, K, 1)).reshape(-1)
+        js = np.arange(rows) % Nw
+        t = time.perf_counter()
+        oracle.matmul_entries(X, "bf16", wp, wa, None, 1, Nw, K, BLOCK, "nf4",
+                              np.zeros(rows, np.int64), js)
+        el = time.perf_counter() - t
+        return el / rows * (M * N)
+
+    for K, N in GEMV_SHAPES:
+        full_time += mm_rows(K, N, 1, 2048)
+        detail[f"gemv_4bit_{K}x{N}"] = "2048 output entries"
+    for K, N in SMALLM_SHAPES:
+        full_time += mm_rows(K, N, SMALLM_M, 2048)
+        detail[f"gemm_4bit_M{SMALLM_M}_{K}x{N}"] = "2048 output entries"
+    M, K, N = PREFILL
+    full_time += mm_rows(K, N, M, 2048)
+    full_time += mm_rows(K, N, M, 16384, backward=True)
+    detail["prefill"] = "2048 forward and 16384 backward output entries (64-row weight slice)"
+    step_bytes = sum(b for _, b, _ in ops)
+    return step_bytes / full_time / 1e9, full_time, detail
+
+
+def cpu_baseline(seconds):
+    gbs, full_s, detail = oracle_sample(seconds)
+    return {"value": round(gbs, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": ("single-threaded C oracle on slices of every op (2^24 quantize/"
+                       "dequantize elements, 2048-16384 output entries per matmul), scaled to the "
+                       f"full step: {round(full_s, 1)} s per step extrapolated"),
+            "host_nproc": os.cpu_count()}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, timed on bounded samples of the workload."""
+    for _ in range(args.warmup):
+        oracle_sample(1.0)
+    t = time.perf_counter()
+    vals = []
+    for _ in range(args.steps):
+        gbs, full_s, _ = oracle_sample(1.0)
+        vals.append(gbs)
+    wall = time.perf_counter() - t
+    v = statistics.mean(vals)
+    base = cpu_baseline(1.0)
+    base["value"] = round(v, 6)
+    return {"metric": METRIC, "value": round(v, 6), "unit": "GB/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "n_elems": N_ELEMS, "quant_type": "nf4",
+                       "blocksize": BLOCK},
+            "cpu_baseline": base,
+            "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    args.cpu_baseline = args.cpu_baseline and rank == 0 and world == 1
+    line = run_ours(args, rank, world, dev)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -129,6 +129,14 @@ def quantize_4bit(x, blocksize: int = 64, quant_type="nf4", stream=None):
     return packed, absmax
 
 
+def quantize_4bit_into(x, packed, absmax, blocksize: int = 64, quant_type="nf4", stream=None):
+    """quantize_4bit into caller-provided outputs (no allocation)."""
+    _need_cuda(x, packed, absmax)
+    _check(bnb4_quantize(_ptr(x), _ptr(packed), _ptr(absmax), x.numel(), blocksize,
+                         _qtype(quant_type), _dtype_code(x), _stream(stream)), "bnb4_quantize")
+    return packed, absmax
+
+
 def dequantize_4bit(packed, absmax, n: int, blocksize: int = 64, quant_type="nf4",
                     dtype=None, out=None, stream=None):
     """-> out[n] of dtype (default bfloat16)."""

@@ -127,6 +127,7 @@ bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *ab
                                bnb4_dtype dt, cudaStream_t stream) {
     bnb4_status s = check_matmul(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt);
     if (s != BNB4_OK) return s;
+    if (N % 8 != 0) return BNB4_ERR_SHAPE;  // dY rows are TMA-loaded: 16-byte row pitch
     return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true, stream));
 }
 

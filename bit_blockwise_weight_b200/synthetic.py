@@ -20,15 +20,21 @@ TORCH_DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat
 
 
 def normal(shape, seed: int, sigma: float = 1.0, dtype: str = "f32",
-           outlier_frac: float = 0.0, outlier_scale: float = 20.0) -> torch.Tensor:
-    """A CPU tensor of the given shape and dtype, drawn as described above."""
-    g = torch.Generator(device="cpu")
+           outlier_frac: float = 0.0, outlier_scale: float = 20.0,
+           device: str = "cpu") -> torch.Tensor:
+    """A tensor of the given shape and dtype, drawn as described above.
+
+    The generator lives on `device`; CPU and CUDA generators give different
+    (each reproducible) streams, so inputs that the CPU oracle must see are
+    drawn on the CPU.
+    """
+    g = torch.Generator(device=device)
     g.manual_seed(int(seed))
-    x = torch.randn(shape, generator=g, dtype=torch.float32)
+    x = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
     if sigma != 1.0:
         x.mul_(sigma)
     if outlier_frac > 0.0:
-        mask = torch.rand(x.numel(), generator=g) < outlier_frac
+        mask = torch.rand(x.numel(), generator=g, device=device) < outlier_frac
         x.view(-1)[mask] *= outlier_scale
     return x.to(TORCH_DTYPES[dtype])
 
@@ -50,9 +56,9 @@ def grad_output(M: int, N: int, seed: int = 3, dtype: str = "bf16") -> torch.Ten
     return normal((M, N), seed, 1.0, dtype)
 
 
-def roundtrip_tensor(n: int, seed: int, dtype: str) -> torch.Tensor:
+def roundtrip_tensor(n: int, seed: int, dtype: str, device: str = "cpu") -> torch.Tensor:
     """1-D N(0, 1) tensor with 1% of the entries scaled by 20 (outliers)."""
-    return normal((n,), seed, 1.0, dtype, outlier_frac=0.01, outlier_scale=20.0)
+    return normal((n,), seed, 1.0, dtype, outlier_frac=0.01, outlier_scale=20.0, device=device)
 
 
 def storage_numpy(t: torch.Tensor):

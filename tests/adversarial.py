@@ -102,3 +102,40 @@ def double_rounding_pairs(qtype: str, out_dtype: str, want: int = 8, seed: int =
             if len(pairs) >= want:
                 return pairs
     return pairs
+
+
+def threshold_neighbourhoods(qtype: str, blocksize: int = 64, n_scales: int = 2048,
+                             radius: int = 4, seed: int = 0):
+    """Blocks [a, x, x, ...] where every x lies within `radius` fp32 steps of a
+    decision threshold scaled by a, for n_scales absmax values a spread over
+    the whole exponent range.  Returns a float32 array of whole blocks."""
+    rng = np.random.default_rng(seed)
+    vals = sorted(set(float(c) for c in bf.table(qtype)))
+    mids = np.array([(p + q) / 2 for p, q in zip(vals, vals[1:])], np.float64)  # exact
+    exps = rng.integers(-126, 128, size=n_scales)
+    exps[:8] = [-126, -97, -96, -95, 95, 96, 97, 127]
+    mant = rng.uniform(1.0, 2.0, size=n_scales)
+    a = (mant * np.exp2(exps.astype(np.float64))).astype(np.float32)
+    a = a[np.isfinite(a) & (a > 0)]
+    xs = []
+    for ai in a:
+        x0 = (mids * np.float64(ai)).astype(np.float32)   # exact product, one rounding
+        cand = [x0]
+        up, dn = x0.copy(), x0.copy()
+        for _ in range(radius):
+            up = np.nextafter(up, np.float32(np.inf))
+            dn = np.nextafter(dn, np.float32(-np.inf))
+            cand += [up, dn]
+        c = np.concatenate(cand)
+        c = c[np.abs(c) <= ai]
+        xs.append((ai, c))
+    per = blocksize - 1
+    blocks = []
+    for ai, c in xs:
+        for j in range(0, c.size, per):
+            blk = np.zeros(blocksize, np.float32)
+            blk[0] = ai
+            part = c[j:j + per]
+            blk[1:1 + part.size] = part
+            blocks.append(blk)
+    return np.concatenate(blocks)

@@ -103,3 +103,65 @@ def test_gemm_small_m_70b_shapes_sampled(q, dt, K, N):
         ref = _ref_forward(Wt, Xs, dt, None, rows)
         err = rel_l2(as_f64(Y, dt).reshape(M, N)[:, rows], ref)
         assert err <= MATMUL_TOL, (M, err)
+
+
+# ---------------------------------------------- large-M gemm and backward (tcgen05)
+
+def _ref_backward(Wt, dYs, dt, M, entries=None):
+    if entries is None:
+        return oracle.matmul_backward(dYs, dt, Wt.packed, Wt.absmax, M, Wt.N, Wt.K, Wt.B, Wt.q)
+    ms, ks = entries
+    return oracle.matmul_backward_entries(dYs, dt, Wt.packed, Wt.absmax, M, Wt.N, Wt.K, Wt.B,
+                                          Wt.q, ms, ks)
+
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N,K,B", [(17, 256, 256, 64), (100, 320, 512, 64), (256, 512, 1024, 128),
+                                     (300, 96, 256, 256), (257, 264, 704, 64)])
+def test_gemm_large_m(q, dt, M, N, K, B):
+    Wt = Weight(N, K, B, q, seed=M)
+    Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
+    bs = synthetic.storage_numpy(synthetic.bias(N, seed=2, dtype=dt)) if M % 2 == 0 else None
+    Y = bnb4.gemm_4bit(to_dev(Xs, dt).view(M, K), Wt.dp, Wt.da, N,
+                       None if bs is None else to_dev(bs, dt), B, q)
+    ref = _ref_forward(Wt, Xs, dt, bs)
+    err = rel_l2(as_f64(to_host(Y), dt).reshape(M, N), ref)
+    assert err <= MATMUL_TOL, err
+
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N,K,B", [(1, 256, 256, 64), (17, 256, 512, 64), (256, 200, 256, 64),
+                                     (300, 320, 768, 256), (64, 1024, 1280, 128)])
+def test_gemm_backward(q, dt, M, N, K, B):
+    Wt = Weight(N, K, B, q, seed=N)
+    dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3, dtype=dt)).reshape(-1)
+    dX = bnb4.gemm_4bit_backward(to_dev(dYs, dt).view(M, N), Wt.dp, Wt.da, K, B, q)
+    ref = _ref_backward(Wt, dYs, dt, M)
+    err = rel_l2(as_f64(to_host(dX), dt).reshape(M, K), ref)
+    assert err <= MATMUL_TOL, err
+
+
+@pytest.mark.parametrize("M", [512, 2048])
+def test_prefill_and_backward_full_size_sampled(M):
+    """M in {512, 2048}, K=4096, N=14336, NF4 B=64, bf16: sampled outputs of both passes."""
+    K, N = 4096, 14336
+    Wt = Weight(N, K, 64, "nf4", seed=0, sigma=0.02)
+    rng = np.random.default_rng(M)
+    Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1)).reshape(-1)
+    Y = as_f64(to_host(bnb4.gemm_4bit(to_dev(Xs, "bf16").view(M, K), Wt.dp, Wt.da, N)),
+               "bf16").reshape(M, N)
+    ms = np.concatenate([[0, M - 1, M - 1], rng.integers(0, M, 509)])
+    js = np.concatenate([[0, N - 1, 0], rng.integers(0, N, 509)])
+    ref = oracle.matmul_entries(Xs, "bf16", Wt.packed, Wt.absmax, None, M, N, K, 64, "nf4", ms, js)
+    err = rel_l2(Y[ms, js], ref)
+    assert err <= MATMUL_TOL, ("forward", err)
+    dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3)).reshape(-1)
+    dX = as_f64(to_host(bnb4.gemm_4bit_backward(to_dev(dYs, "bf16").view(M, N), Wt.dp, Wt.da, K)),
+                "bf16").reshape(M, K)
+    ks = np.concatenate([[0, K - 1, 0], rng.integers(0, K, 253)])
+    ms2 = ms[:ks.size]
+    refb = _ref_backward(Wt, dYs, "bf16", M, (ms2, ks))
+    err = rel_l2(dX[ms2, ks], refb)
+    assert err <= MATMUL_TOL, ("backward", err)

@@ -55,6 +55,20 @@ def test_division_knife_edges(q):
 
 
 @pytest.mark.parametrize("q", ["nf4", "fp4"])
+def test_quotients_next_to_every_threshold(q):
+    """x within 4 fp32 steps of every decision threshold times a, for 2048 absmax
+    values over the whole exponent range (both sides of the reciprocal path's
+    range limits included)."""
+    import adversarial
+    blk = adversarial.threshold_neighbourhoods(q, 64, n_scales=2048, radius=4, seed=11)
+    gp, ga = _gpu_quant(blk, "f32", 64, q)
+    op, oa = oracle.quantize(blk, "f32", 64, q)
+    assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32))
+    bad = np.nonzero(gp != op)[0]
+    assert bad.size == 0, (bad.size, bad[:4])
+
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
 @pytest.mark.parametrize("out", ["bf16", "f16"])
 def test_dequant_double_rounding_edges(q, out):
     import adversarial

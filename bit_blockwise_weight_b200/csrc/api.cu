@@ -109,7 +109,11 @@ bnb4_status bnb4_gemv(const void *x, const uint8_t *W, const float *absmax, cons
                       bnb4_dtype dt, cudaStream_t stream) {
     bnb4_status s = check_matmul(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt);
     if (s != BNB4_OK) return s;
-    return from_cuda(launch_gemv(x, W, absmax, bias, y, N, K, blocksize, qt, dt, stream));
+    if (N <= gemv_max_rows() && K <= gemv_max_k())
+        return from_cuda(launch_gemv(x, W, absmax, bias, y, N, K, blocksize, qt, dt, stream));
+    // shapes beyond the CUDA-core kernel's shared-memory plan: the same product
+    // through the matrix kernels (x is a 1 x K matrix)
+    return bnb4_gemm(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt, stream);
 }
 
 bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, const void *bias,
@@ -117,7 +121,9 @@ bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, cons
                       bnb4_dtype dt, cudaStream_t stream) {
     bnb4_status s = check_matmul(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt);
     if (s != BNB4_OK) return s;
-    if (M <= kSmallMMax)
+    // small M streams the weight once per call; the per-CTA row range of that
+    // kernel is capped at 1024 rows, beyond which the tensor-core kernel takes over
+    if (M <= kSmallMMax && N <= (int64_t)device_sm_count() * 1024)
         return from_cuda(launch_gemm_small(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, stream));
     return from_cuda(launch_gemm_tc(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, false, stream));
 }

@@ -14,48 +14,34 @@
 // replicated once per shared-memory bank (32 KB) so that every lane reads its
 // own bank: lookups never conflict.
 //
-// K order inside a 128-element span: lane (g, t) owns weights [32t, 32t+32)
-// of rows g and g+8 (16 contiguous bytes each).  For mma step s it feeds
-// bytes 2s and 2s+1 of its chunk, so k-slot 2t+e holds k = 32t + 4s + e and
-// k-slot 2t+8+e holds k = 32t + 4s + 2 + e; the B fragment takes the same k
-// values of X.  The reduction over k is a plain sum, so this order is free.
+// K order inside a 64-element quantization block: lane (g, t) owns weights
+// [16t, 16t+16) of rows g and g+8 (8 contiguous bytes each).  For mma step s
+// (0..3) it feeds bytes 2s and 2s+1 of its 8, so k-slot 2t+e holds
+// k = 16t + 4s + e and k-slot 2t+8+e holds k = 16t + 4s + 2 + e; the B
+// fragment takes the same k values of X.  The reduction over k is a plain sum,
+// so the order is free, and every step stays inside one block: the four steps
+// of a block accumulate into a block sum that is scaled by the block's absmax
+// in fp32 once.
 //
-// absmax: with blocksize 64 a span holds two blocks (lanes t < 2 carry block
-// 0, t >= 2 block 1).  Two mma per step, each with the other block's B values
-// zeroed, keep the two block sums apart; each is scaled by its absmax in fp32.
-// For blocksize >= 128 a span lies in one block and one mma per step does.
-//
-// CTA: 4 warps on 32 rows; a 512-element window of K per iteration (one span
-// per warp), X windows double-buffered in shared memory with cp.async, weight
-// chunks double-buffered in registers.  Warps' partial sums meet in shared
-// memory; K split over a thread-block cluster meets in distributed shared
-// memory.  No global scratch.
-#include <cooperative_groups.h>
-
+// Work split (persistent, one CTA per SM): CTA c owns rows
+// [N c / G, N (c+1) / G) -- balanced to one row -- and all of K.  Its rows form
+// T tiles of 16 (the last one partial), grouped by up to 4 per warp so that
+// each X fragment feeds 4 tiles; the 8 warps split the groups and then K.
+// Weights, absmax and X fragments of the next block are loaded into registers
+// while the current block is multiplied.  Partial sums of the warps that
+// share a group meet in shared memory.  No global scratch.
 #include "common.cuh"
 #include "kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace bnb4 {
 
 namespace {
 
-constexpr int kWarps = 4;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kRows = 32;              // rows of W per CTA (two m16 tiles)
-constexpr int kSpan = 128;             // K elements per warp per window
-constexpr int kWin = kWarps * kSpan;   // 512
-constexpr int kXStride = kWin + 16;    // bf16 elements per X row in smem (+32 B: no bank conflicts)
+constexpr int MT = 4;                 // m16 tiles per warp
+constexpr int kMaxTiles = 64;         // rows per CTA <= 1024
 constexpr int kMaxM = 16;
-
-__device__ __forceinline__ uint4 ld_stream(const uint8_t *p) {
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
 
 template <typename D> struct Mma;
 template <> struct Mma<BF16> {
@@ -75,8 +61,11 @@ template <> struct Mma<F16> {
     }
 };
 
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ uint2 ld_stream8(const uint8_t *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
 
 // byte j (0..3) of a word -> offset of its entry in this lane's bank
 // (entry e of lane l sits at word 32 e + l)
@@ -85,288 +74,205 @@ __device__ __forceinline__ uint32_t lut_off(uint32_t w, int j, uint32_t lane4) {
     return (sh & 0x7f80u) | lane4;
 }
 
-__device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
-    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(s), "l"(gmem));
-}
-
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 
+struct Frag {
+    uint2 w[MT][2];     // rows g and g+8 of each tile: 8 bytes (16 weights)
+    float a[MT][2];     // their block absmax
+};
+
 template <typename D, int NT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 gemm_small_kernel(const uint16_t *__restrict__ X, const uint8_t *__restrict__ W,
                   const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-                  uint16_t *__restrict__ Y, int M, int N, int K, int log2B, int Kc,
-                  CodeTable tab) {
+                  uint16_t *__restrict__ Y, int M, int N, int K, int log2B, CodeTable tab) {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);                        // 256 x 32 words
-    uint16_t *xwin = reinterpret_cast<uint16_t *>(smem + 256 * 32 * 4);        // [2][16][kXStride]
-    float *red = reinterpret_cast<float *>(xwin + 2 * kMaxM * kXStride);       // [kWarps][32][16]
+    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);                 // 256 x 32 words
+    float *sum = reinterpret_cast<float *>(smem + 256 * 32 * 4);        // [kMaxTiles*16][16]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int ksplit = gridDim.y;
-    const int k0 = blockIdx.y * Kc;
-    const int k1 = min(K, k0 + Kc);
-    const int row0 = blockIdx.x * kRows;
+
+    // CTA rows
+    const int G = gridDim.x;
+    const int r0 = (int)(((int64_t)N * blockIdx.x) / G);
+    const int r1 = (int)(((int64_t)N * (blockIdx.x + 1)) / G);
+    const int T = (r1 - r0 + 15) >> 4;  // tiles
+    const int nb = K >> 6;              // 64-element blocks along K
     const int64_t row_bytes = K >> 1;
     const int nblk = K >> log2B;
 
-    // byte -> code pair table, one copy per bank
-    for (int e = tid; e < 256; e += kThreads) {
+    // byte -> code pair table, one copy per bank (a thread fills 4 copies at once)
+    for (int e = tid >> 3; e < 256; e += kThreads / 8) {
         const uint32_t v = Dt<D>::pack2(tab.v[e >> 4], tab.v[e & 15]);
-#pragma unroll 4
-        for (int b = 0; b < 32; ++b) lut[e * 32 + b] = v;
+        reinterpret_cast<uint4 *>(lut + e * 32)[tid & 7] = make_uint4(v, v, v, v);
     }
-
-    const int nwin = (k1 - k0 + kWin - 1) / kWin;
-    // X window in the order the B fragments read it: the group of 4 elements
-    // k = 128 w + 32 t + 4 s (+0..3) sits at 128 w + 16 s + 4 t, so the four
-    // lanes t of one step read 32 contiguous bytes
-    auto load_xwin = [&](int wi, int buf) {
-        const int kb = k0 + wi * kWin;
-        uint16_t *dst = xwin + buf * kMaxM * kXStride;
-        for (int c = tid; c < M * (kWin / 4); c += kThreads) {
-            const int m = c / (kWin / 4), q = c % (kWin / 4);
-            const int k = kb + q * 4;
-            const int w = q >> 5, tt = (q >> 3) & 3, ss = q & 7;
-            uint16_t *d = dst + m * kXStride + w * kSpan + ss * 16 + tt * 4;
-            if (k < k1)
-                cp_async8(d, X + (int64_t)m * K + k);
-            else
-                *reinterpret_cast<uint2 *>(d) = make_uint2(0, 0);
-        }
-        cp_async_commit();
-    };
-    // rows >= M of both X buffers stay zero
-    for (int c = tid; c < 2 * kMaxM * kXStride / 8; c += kThreads) {
-        const int m = (c * 8 / kXStride) % kMaxM;
-        if (m >= M) reinterpret_cast<uint4 *>(xwin)[c] = make_uint4(0, 0, 0, 0);
-    }
-
-    // this lane's rows: tile mt, half h -> row0 + 16 mt + 8 h + g
-    int rows[2][2];
-    bool rv[2][2];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            rows[mt][h] = row0 + 16 * mt + 8 * h + g;
-            rv[mt][h] = rows[mt][h] < N;
-        }
-    auto load_w = [&](int wi, uint4 (&dst)[2][2]) {
-        const int kk = k0 + wi * kWin + warp * kSpan + 32 * t;
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                dst[mt][h] = (rv[mt][h] && kk < k1)
-                                 ? ld_stream(W + (int64_t)rows[mt][h] * row_bytes + (kk >> 1))
-                                 : make_uint4(0, 0, 0, 0);
-    };
-
-    float acc[2][NT][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
+    for (int e = tid; e < T * 16 * kMaxM; e += kThreads) sum[e] = 0.f;
+    __syncthreads();
+    if (T == 0) return;
 
     const uint32_t lut_base = (uint32_t)__cvta_generic_to_shared(lut);
     const uint32_t lane4 = 4u * lane;
-    const bool two_blocks = log2B == 6;  // blocksize 64: a span holds two blocks
 
-    uint4 wcur[2][2], wnxt[2][2];
-    if (nwin > 0) {
-        load_xwin(0, 0);
-        load_w(0, wcur);
-    }
-    __syncthreads();  // lut ready
+    // warp -> (tile group, K part)
+    const int groups = (T + MT - 1) / MT;
+    for (int gbase = 0; gbase < groups; gbase += kWarps) {
+        const int gcount = min(kWarps, groups - gbase);
+        const int kparts = kWarps / gcount;
+        const int gi = gbase + warp / kparts;
+        const int kp = warp % kparts;
+        const bool active = warp < gcount * kparts;
+        const int b_lo = active ? (int)(((int64_t)nb * kp) / kparts) : 0;
+        const int b_hi = active ? (int)(((int64_t)nb * (kp + 1)) / kparts) : 0;
 
-    for (int wi = 0; wi < nwin; ++wi) {
-        cp_async_wait_all();
-        __syncthreads();  // X window wi visible; the other buffer is free
-        if (wi + 1 < nwin) {
-            load_xwin(wi + 1, (wi + 1) & 1);
-            load_w(wi + 1, wnxt);
-        }
-        const int kspan = k0 + wi * kWin + warp * kSpan;
-        const uint16_t *xb = xwin + (wi & 1) * kMaxM * kXStride + warp * kSpan + 4 * t;
-
-        float plo[2][NT][4], phi[2][NT][4];
+        int rows[MT][2];
+        bool rv[MT][2];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) plo[mt][nt][i] = phi[mt][nt][i] = 0.f;
-
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-            uint32_t b[NT][2];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const uint2 v = *reinterpret_cast<const uint2 *>(xb + (nt * 8 + g) * kXStride + 16 * s);
-                b[nt][0] = v.x;
-                b[nt][1] = v.y;
-            }
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                const uint32_t wg = (&wcur[mt][0].x)[s >> 1];
-                const uint32_t wg8 = (&wcur[mt][1].x)[s >> 1];
-                const int j0 = 2 * (s & 1), j1 = j0 + 1;
-                uint32_t a[4];
-                a[0] = lds32(lut_base + lut_off(wg, j0, lane4));
-                a[1] = lds32(lut_base + lut_off(wg8, j0, lane4));
-                a[2] = lds32(lut_base + lut_off(wg, j1, lane4));
-                a[3] = lds32(lut_base + lut_off(wg8, j1, lane4));
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    if (two_blocks) {
-                        const uint32_t lo0 = t < 2 ? b[nt][0] : 0u, lo1 = t < 2 ? b[nt][1] : 0u;
-                        const uint32_t hi0 = t < 2 ? 0u : b[nt][0], hi1 = t < 2 ? 0u : b[nt][1];
-                        Mma<D>::run(plo[mt][nt], a, lo0, lo1);
-                        Mma<D>::run(phi[mt][nt], a, hi0, hi1);
-                    } else {
-                        Mma<D>::run(plo[mt][nt], a, b[nt][0], b[nt][1]);
-                    }
-                }
-            }
-        }
-        // block scales: rows g / g+8 of each tile, blocks of k = kspan and kspan + 64
-        const int blo = kspan >> log2B;
-        const int bhi = (kspan + 64) >> log2B;
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            float alo[2], ahi[2];
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const float *ap = absmax + (int64_t)rows[mt][h] * nblk;
-                alo[h] = (rv[mt][h] && kspan < k1) ? __ldg(ap + blo) : 0.f;
-                ahi[h] = (rv[mt][h] && two_blocks && kspan + 64 < k1) ? __ldg(ap + bhi) : 0.f;
+                rows[mt][h] = r0 + 16 * (gi * MT + mt) + 8 * h + g;
+                rv[mt][h] = active && (gi * MT + mt) < T && rows[mt][h] < r1;
             }
+        auto fetch = [&](int b, Frag &f) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if (rv[mt][h]) {
+                        const int64_t rb = (int64_t)rows[mt][h];
+                        f.w[mt][h] = ld_stream8(W + rb * row_bytes + 32 * b + 8 * t);
+                        f.a[mt][h] = __ldg(absmax + rb * nblk + ((64 * b) >> log2B));
+                    } else {
+                        f.w[mt][h] = make_uint2(0, 0);
+                        f.a[mt][h] = 0.f;
+                    }
+                }
+        };
+        // X fragment of block b: lane (g, t) needs X[nt*8 + g][64b + 16t + 4s .. +4] for s = 0..3
+        auto fetch_x = [&](int b, uint2 (&xf)[4][NT]) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int m = nt * 8 + g;
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    xf[s][nt] = (m < M) ? __ldg(reinterpret_cast<const uint2 *>(
+                                              X + (int64_t)m * K + 64 * b + 16 * t + 4 * s))
+                                        : make_uint2(0, 0);
+            }
+        };
+
+        float acc[MT][NT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int h = i >> 1;
-                    acc[mt][nt][i] = __fmaf_rn(plo[mt][nt][i], alo[h], acc[mt][nt][i]);
-                    if (two_blocks) acc[mt][nt][i] = __fmaf_rn(phi[mt][nt][i], ahi[h], acc[mt][nt][i]);
-                }
+                for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
+
+        Frag cur, nxt;
+        uint2 xc[4][NT], xn[4][NT];
+        if (b_lo < b_hi) {
+            fetch(b_lo, cur);
+            fetch_x(b_lo, xc);
         }
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) wcur[mt][h] = wnxt[mt][h];
-    }
-
-    // warps' partial sums -> red[warp][row][m]
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = 16 * mt + 8 * (i >> 1) + g;
-                const int m = nt * 8 + 2 * t + (i & 1);
-                red[(warp * kRows + r) * kMaxM + m] = acc[mt][nt][i];
+        for (int b = b_lo; b < b_hi; ++b) {
+            if (b + 1 < b_hi) {
+                fetch(b + 1, nxt);
+                fetch_x(b + 1, xn);
             }
-    __syncthreads();
-    for (int e = tid; e < kRows * kMaxM; e += kThreads) {
-        float v = 0.f;
+            float blk[MT][NT][4];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += red[w * kRows * kMaxM + e];
-        red[e] = v;  // red[0] now holds the CTA's sums (each e read only by its owner)
-    }
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) blk[mt][nt][i] = 0.f;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const int wi = s >> 1, j0 = 2 * (s & 1), j1 = j0 + 1;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const uint32_t wg = wi ? cur.w[mt][0].y : cur.w[mt][0].x;
+                    const uint32_t wg8 = wi ? cur.w[mt][1].y : cur.w[mt][1].x;
+                    uint32_t a[4];
+                    a[0] = lds32(lut_base + lut_off(wg, j0, lane4));
+                    a[1] = lds32(lut_base + lut_off(wg8, j0, lane4));
+                    a[2] = lds32(lut_base + lut_off(wg, j1, lane4));
+                    a[3] = lds32(lut_base + lut_off(wg8, j1, lane4));
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) Mma<D>::run(blk[mt][nt], a, xc[s][nt].x, xc[s][nt].y);
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        acc[mt][nt][i] = __fmaf_rn(blk[mt][nt][i], cur.a[mt][i >> 1], acc[mt][nt][i]);
+            cur = nxt;
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) xc[s][nt] = xn[s][nt];
+        }
 
-    auto finish = [&](int e, float v) {
+        // this warp's partial sums -> shared sums (warps of a group split K)
+        if (active) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int tile = gi * MT + mt;
+                if (tile >= T) continue;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int r = 16 * tile + 8 * (i >> 1) + g;
+                        const int m = nt * 8 + 2 * t + (i & 1);
+                        if (m < M) atomicAdd(&sum[r * kMaxM + m], acc[mt][nt][i]);
+                    }
+            }
+        }
+    }
+    __syncthreads();
+    for (int e = tid; e < T * 16 * kMaxM; e += kThreads) {
         const int r = e / kMaxM, m = e % kMaxM;
-        const int row = row0 + r;
-        if (m < M && row < N) {
+        const int row = r0 + r;
+        if (m < M && row < r1) {
+            float v = sum[e];
             if (bias) v += Dt<D>::to_f32(bias[row]);
             Y[(int64_t)m * N + row] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);
         }
-    };
-
-    if (ksplit == 1) {
-        __syncthreads();
-        for (int e = tid; e < kRows * kMaxM; e += kThreads) finish(e, red[e]);
-        return;
     }
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const int rank = (int)cluster.block_rank();
-    for (int e = tid; e < kRows * kMaxM; e += kThreads) {
-        if (e % ksplit != rank) continue;
-        float v = 0.f;
-        for (int q = 0; q < ksplit; ++q) v += *cluster.map_shared_rank(&red[e], q);
-        finish(e, v);
-    }
-    cluster.sync();
 }
 
-size_t smem_bytes() {
-    return 256 * 32 * 4 + 2 * kMaxM * kXStride * 2 + kWarps * kRows * kMaxM * 4;
-}
-
-// choose the K split (cluster size) that fills the GPU's CTA slots most evenly
-int pick_ksplit(int groups, int wins, int slots) {
-    int best = 1;
-    double best_eff = 0.0;
-    for (int ks = 1; ks <= 8 && ks <= wins; ++ks) {
-        const int per = (wins + ks - 1) / ks;
-        const int ks_eff = (wins + per - 1) / per;
-        if (ks_eff != ks) continue;
-        const long units = (long)groups * ks;
-        const long waves = (units + slots - 1) / slots;
-        const double eff = (double)units / (double)(waves * slots) * (1.0 - 0.02 * (ks - 1));
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
-            best = ks;
-        }
-    }
-    return best;
-}
+size_t smem_bytes(int tiles) { return 256 * 32 * 4 + (size_t)tiles * 16 * kMaxM * 4; }
 
 template <typename D, int NT>
 cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const void *bias,
                      void *Y, int M, int N, int K, int log2B, const CodeTable &tab,
                      cudaStream_t stream) {
-    const size_t smem = smem_bytes();
-    static bool attr_set = false;  // benign race: setting it twice is harmless
-    if (!attr_set) {
+    const int G = device_sm_count();
+    const int max_rows = (N + G - 1) / G;
+    const int tiles = (max_rows + 15) / 16;
+    if (tiles > kMaxTiles) return cudaErrorInvalidValue;
+    const size_t smem = smem_bytes(tiles);
+    static int smem_set = 0;  // largest dynamic shared memory size set so far
+    if ((int)smem > 48 * 1024 && (int)smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(gemm_small_kernel<D, NT>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        smem_set = (int)smem;
     }
-    const int groups = (N + kRows - 1) / kRows;
-    const int wins = (K + kWin - 1) / kWin;
-    const int slots = device_sm_count() * 3;
-    const int ks = pick_ksplit(groups, wins, slots);
-    const int per = (wins + ks - 1) / ks;
-    const int Kc = per * kWin;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(groups, ks, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = ks;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT>, static_cast<const uint16_t *>(X), W,
-                              absmax, static_cast<const uint16_t *>(bias),
-                              static_cast<uint16_t *>(Y), M, N, K, log2B, Kc, tab);
+    gemm_small_kernel<D, NT><<<G, kThreads, smem, stream>>>(
+        static_cast<const uint16_t *>(X), W, absmax, static_cast<const uint16_t *>(bias),
+        static_cast<uint16_t *>(Y), M, N, K, log2B, tab);
+    return cudaGetLastError();
 }
 
 }  // namespace

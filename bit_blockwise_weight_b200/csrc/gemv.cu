@@ -4,177 +4,248 @@
 // dequant + dot kernel; the bias epilogue is added before the one rounding of
 // the output (section Correctness).  The weight stream (0.5 B per weight plus
 // 4 B of absmax per block) is the whole cost, so the kernel is built around
-// reading it once, coalesced, with enough bytes in flight.
+// reading it once, coalesced, with enough bytes in flight and as few
+// shared-memory wavefronts per weight as possible.
 //
-// Work split:
-//   * a CTA (8 warps) owns 32 rows and a K-range; warp w owns 4 rows;
-//   * lane l reads 16 packed bytes (32 weights) of each of its warp's 4 rows
-//     per 1024-element segment -- 512 contiguous bytes per row per warp load;
-//   * x of the CTA's K-range is converted once to fp32 in shared memory;
-//   * each lane decodes nibbles through a 16-entry code table held in the
-//     warp's lanes (shfl), accumulates sum_k code * x in fp32 over its 32
-//     weights (all inside one quantization block) and scales by the block's
-//     absmax once;
-//   * rows are reduced across lanes with xor-shuffles;
-//   * when K is split over CTAs, the CTAs of one row range form a thread-block
-//     cluster and add their partial rows through distributed shared memory,
-//     so no global scratch is needed.
-#include <cooperative_groups.h>
-
+// Work split (persistent, one CTA per SM):
+//   * CTA c owns rows [N c / G, N (c+1) / G) (balanced to one row) and all of
+//     K; x is copied once into shared memory (16-bit, swizzled so that the
+//     per-lane reads below never conflict);
+//   * the CTA's work is a list of units (quad of 4 rows, 1024-element segment
+//     of K), split into 16 equal contiguous ranges, one per warp;
+//   * lane l of a warp owns 32 weights (16 packed bytes) of each row of the
+//     unit: 512 contiguous bytes per row per warp;
+//   * every lane streams its own bytes (and their block absmax) through a
+//     3-slot cp.async ring in shared memory, so two units are in flight per
+//     warp without holding registers;
+//   * decode: a 256-entry table, replicated once per bank, maps a packed byte
+//     to its two codes as a bf16x2 / f16x2 word (one conflict-free lookup per
+//     two weights); each code is multiplied by x with a mixed-precision FMA
+//     (16-bit operands, fp32 accumulate), so nothing is unpacked;
+//   * the lane's 32 weights lie in one quantization block: their sum is
+//     scaled by the block absmax once, in fp32;
+//   * when a warp leaves a quad, its 4 row sums are reduced across lanes with
+//     xor-shuffles and added to the CTA's row sums in shared memory.
+// The codes enter as 16-bit values (the code table rounded once to bf16 /
+// fp16), like the weight operand of the tensor-core kernels.  No global
+// scratch.
 #include "common.cuh"
 #include "kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace bnb4 {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kRowsPerWarp = 4;
-constexpr int kRowsPerCta = kWarps * kRowsPerWarp;  // 32
-constexpr int kSeg = 1024;                          // elements per warp-wide load
-constexpr int kMaxKc = 8192;                        // fp32 x slice <= 32 KB
+constexpr int kWarps = 16;
+constexpr int kThreads = kWarps * 32;
+constexpr int kSeg = 1024;       // elements per unit per row (32 lanes x 32)
+constexpr int STAGES = 3;
+constexpr int kSlot = 4 * 32 * 16 + 32 * 16;  // W [4 rows][32 lanes] 16 B + absmax [32 lanes][4]
+constexpr int kLut = 256 * 32 * 4;            // 32 KB
+constexpr int kMaxRows = 1024;   // rows per CTA
+constexpr int kMaxK = 32768;
 
-__device__ __forceinline__ uint32_t shfl_idx(uint32_t v, uint32_t lane_bits) {
-    uint32_t r;
-    asm volatile("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;"
-                 : "=r"(r)
-                 : "r"(v), "r"(lane_bits));
-    return r;
-}
-
-__device__ __forceinline__ uint4 ld_stream(const uint8_t *p) {
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
+                 : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
 }
 
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void *src, bool valid) {
+    const int n = valid ? BYTES : 0;
+    if (BYTES == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n));
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;" ::"r"(dst), "l"(src),
+                     "n"(BYTES), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// acc += code.lo * x.lo + code.hi * x.hi with 16-bit operands and an fp32 accumulator
+template <typename D> struct Fma2;
+template <> struct Fma2<BF16> {
+    __device__ static __forceinline__ void run(float &a0, float &a1, uint32_t c, uint32_t x) {
+        asm("{\n\t.reg .b16 c0, c1, x0, x1;\n\t"
+            "mov.b32 {c0, c1}, %2;\n\tmov.b32 {x0, x1}, %3;\n\t"
+            "fma.rn.f32.bf16 %0, c0, x0, %0;\n\tfma.rn.f32.bf16 %1, c1, x1, %1;\n\t}"
+            : "+f"(a0), "+f"(a1)
+            : "r"(c), "r"(x));
+    }
+};
+template <> struct Fma2<F16> {
+    __device__ static __forceinline__ void run(float &a0, float &a1, uint32_t c, uint32_t x) {
+        asm("{\n\t.reg .b16 c0, c1, x0, x1;\n\t"
+            "mov.b32 {c0, c1}, %2;\n\tmov.b32 {x0, x1}, %3;\n\t"
+            "fma.rn.f32.f16 %0, c0, x0, %0;\n\tfma.rn.f32.f16 %1, c1, x1, %1;\n\t}"
+            : "+f"(a0), "+f"(a1)
+            : "r"(c), "r"(x));
+    }
+};
+
+// element k of x -> its 16-bit slot in shared memory.  Lane chunks of 32
+// elements (64 B) hold four 16-byte pieces; piece i of chunk L sits at
+// position i ^ ((L >> 1) & 3), which spreads the eight lanes of a quarter
+// warp over all 32 banks.
+__device__ __forceinline__ int xswz(int k) {
+    const int L = k >> 5, i = (k >> 3) & 3;
+    return (L << 5) | ((i ^ ((L >> 1) & 3)) << 3) | (k & 7);
+}
+
 template <typename D>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-            uint16_t *__restrict__ y, int N, int K, int log2B, int Kc, CodeTable tab) {
-    extern __shared__ float xs[];  // [Kc] fp32
-    __shared__ float partial[kRowsPerCta];
+            uint16_t *__restrict__ y, int N, int K, int log2B, CodeTable tab) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
+    uint8_t *ring = smem + kLut;                                                  // warps x STAGES
+    float *rowsum = reinterpret_cast<float *>(ring + kWarps * STAGES * kSlot);    // [kMaxRows]
+    uint16_t *xs = reinterpret_cast<uint16_t *>(rowsum + kMaxRows);              // [K] swizzled
 
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int ksplit = gridDim.y, kpart = blockIdx.y;
-    const int k0 = kpart * Kc;
-    const int k1 = min(K, k0 + Kc);
-    const int row0 = blockIdx.x * kRowsPerCta;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = gridDim.x;
+    const int r0 = (int)(((int64_t)N * blockIdx.x) / G);
+    const int r1 = (int)(((int64_t)N * (blockIdx.x + 1)) / G);
+    const int rows = r1 - r0;
+    const int Q = (rows + 3) >> 2;
+    const int S = (K + kSeg - 1) / kSeg;
+    const int U = Q * S;
+    const int64_t row_bytes = K >> 1;
+    const int nblk = K >> log2B;
 
-    // x slice -> fp32 shared memory
-    for (int k = k0 + threadIdx.x; k < k1; k += blockDim.x) xs[k - k0] = Dt<D>::to_f32(x[k]);
+    for (int e = tid >> 3; e < 256; e += kThreads / 8) {
+        const uint32_t v = Dt<D>::pack2(tab.v[e >> 4], tab.v[e & 15]);
+        reinterpret_cast<uint4 *>(lut + e * 32)[tid & 7] = make_uint4(v, v, v, v);
+    }
+    for (int k = tid; k < K; k += kThreads) xs[xswz(k)] = x[k];
+    for (int r = tid; r < rows; r += kThreads) rowsum[r] = 0.f;
     __syncthreads();
 
-    const uint32_t my_code = __float_as_uint(tab.v[lane & 15]);
-    const int64_t row_bytes = K >> 1;
-    const int nblk = K >> log2B;  // absmax entries per row
+    const uint32_t lut_base = (uint32_t)__cvta_generic_to_shared(lut);
+    const uint32_t lane4 = 4u * lane;
+    const uint32_t my_ring = (uint32_t)__cvta_generic_to_shared(ring) + warp * STAGES * kSlot;
+    const uint32_t xs_base = (uint32_t)__cvta_generic_to_shared(xs);
+    const int u_lo = (int)(((int64_t)U * warp) / kWarps);
+    const int u_hi = (int)(((int64_t)U * (warp + 1)) / kWarps);
 
-    int rows[kRowsPerWarp];
-    bool rvalid[kRowsPerWarp];
+    auto issue = [&](int u, int slot) {
+        const uint32_t base = my_ring + slot * kSlot;
+        const int q = u / S, s = u - q * S;
+        const int k = s * kSeg + 32 * lane;
+        const bool ok = u < u_hi && k < K;
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        rows[r] = row0 + warp * kRowsPerWarp + r;
-        rvalid[r] = rows[r] < N;
-    }
-
-    float acc[kRowsPerWarp] = {0.f, 0.f, 0.f, 0.f};
-    const int nseg = (k1 - k0 + kSeg - 1) / kSeg;
-
-    // software pipeline: weights of segment s+1 are in flight while s computes
-    uint4 wcur[kRowsPerWarp], wnext[kRowsPerWarp];
-    auto load_seg = [&](int s, uint4 *dst) {
-        const int kk = k0 + s * kSeg + lane * 32;
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-            if (rvalid[r] && kk < k1)
-                dst[r] = ld_stream(W + (int64_t)rows[r] * row_bytes + (kk >> 1));
-            else
-                dst[r] = make_uint4(0, 0, 0, 0);
+        for (int r = 0; r < 4; ++r) {
+            const int row = r0 + 4 * q + r;
+            const bool v = ok && row < r1;
+            cp_async<16>(base + (r * 32 + lane) * 16,
+                         v ? W + (int64_t)row * row_bytes + (k >> 1) : W, v);
+            cp_async<4>(base + 4 * 32 * 16 + lane * 16 + 4 * r,
+                        v ? absmax + (int64_t)row * nblk + (k >> log2B) : absmax, v);
         }
     };
-    if (nseg > 0) load_seg(0, wcur);
 
-    for (int s = 0; s < nseg; ++s) {
-        if (s + 1 < nseg) load_seg(s + 1, wnext);
-        const int kk = k0 + s * kSeg + lane * 32;
-        const bool kvalid = kk < k1;  // K % 32 == 0: a lane's 32 weights are all in or all out
-        // every lane runs the decode (its shuffles need the whole warp); lanes
-        // past the end multiply zero weights by zero x
-        float xv[32];
-        if (kvalid) {
-            const float4 *xp = reinterpret_cast<const float4 *>(xs + (kk - k0));
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float4 v = xp[q];
-                xv[4 * q] = v.x; xv[4 * q + 1] = v.y; xv[4 * q + 2] = v.z; xv[4 * q + 3] = v.w;
+    for (int i = 0; i < STAGES - 1; ++i) {
+        issue(u_lo + i, i);
+        cp_async_commit();
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int q_cur = U > 0 ? u_lo / S : 0;
+    for (int u = u_lo; u < u_hi; ++u) {
+        const int it = u - u_lo;
+        issue(u + STAGES - 1, (it + STAGES - 1) % STAGES);
+        cp_async_commit();
+        cp_async_wait<STAGES - 1>();
+        const uint32_t base = my_ring + (it % STAGES) * kSlot;
+        const int q = u / S, s = u - q * S;
+        const int k = s * kSeg + 32 * lane;
+        // x[k .. k+32) as 16 bf16x2 / f16x2 words (zeros past the end of K)
+        uint32_t xq[16];
+        if (k < K) {
+            const int L = k >> 5;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = lds128(xs_base + ((L << 5) | ((i ^ ((L >> 1) & 3)) << 3)) * 2);
+                xq[4 * i] = v.x; xq[4 * i + 1] = v.y; xq[4 * i + 2] = v.z; xq[4 * i + 3] = v.w;
             }
         } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) xv[q] = 0.f;
+            for (int i = 0; i < 16; ++i) xq[i] = 0u;
         }
-        const int blk = kk >> log2B;
+        const uint4 av = lds128(base + 4 * 32 * 16 + lane * 16);
+        const float am[4] = {__uint_as_float(av.x), __uint_as_float(av.y), __uint_as_float(av.z),
+                             __uint_as_float(av.w)};
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-            const float a = (rvalid[r] && kvalid) ? __ldg(absmax + (int64_t)rows[r] * nblk + blk) : 0.f;
-            const uint32_t w4[4] = {wcur[r].x, wcur[r].y, wcur[r].z, wcur[r].w};
+        for (int r = 0; r < 4; ++r) {
+            const uint4 wv = lds128(base + (r * 32 + lane) * 16);
+            const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
             float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int qq = 0; qq < 4; ++qq) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const float ch = __uint_as_float(shfl_idx(my_code, w4[q] >> (8 * j + 4)));
-                    const float cl = __uint_as_float(shfl_idx(my_code, w4[q] >> (8 * j)));
-                    s0 = __fmaf_rn(ch, xv[8 * q + 2 * j], s0);
-                    s1 = __fmaf_rn(cl, xv[8 * q + 2 * j + 1], s1);
+                    // byte j of word qq = weights 8qq+2j (high nibble) and 8qq+2j+1
+                    const uint32_t sh = j == 0 ? (w4[qq] << 7) : (w4[qq] >> (8 * j - 7));
+                    const uint32_t c2 = lds32(lut_base + ((sh & 0x7f80u) | lane4));
+                    Fma2<D>::run(s0, s1, c2, xq[4 * qq + j]);
                 }
             }
-            acc[r] = __fmaf_rn(s0 + s1, a, acc[r]);
+            acc[r] = __fmaf_rn(s0 + s1, am[r], acc[r]);
         }
+        // leaving this quad: fold the lane sums into the CTA's row sums
+        if (u + 1 == u_hi || (u + 1) / S != q) {
 #pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) wcur[r] = wnext[r];
-    }
-
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        const float v = warp_sum(acc[r]);
-        if (lane == 0) partial[warp * kRowsPerWarp + r] = v;
-    }
-
-    if (ksplit == 1) {
-        __syncthreads();
-        if (threadIdx.x < kRowsPerCta) {
-            const int row = row0 + threadIdx.x;
-            if (row < N) {
-                float v = partial[threadIdx.x];
-                if (bias) v += Dt<D>::to_f32(bias[row]);
-                y[row] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);
+            for (int r = 0; r < 4; ++r) {
+                const float v = warp_sum(acc[r]);
+                const int row = 4 * q + r;
+                if (lane == 0 && row < rows) atomicAdd(&rowsum[row], v);
+                acc[r] = 0.f;
             }
         }
-        return;
+        (void)q_cur;
     }
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int r = tid; r < rows; r += kThreads) {
+        float v = rowsum[r];
+        if (bias) v += Dt<D>::to_f32(bias[r0 + r]);
+        y[r0 + r] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);
+    }
+}
 
-    // K split over the CTAs of a cluster: rank r finishes rows r, r + ksplit, ...
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
-    const int rank = (int)cluster.block_rank();
-    if (threadIdx.x < kRowsPerCta && (threadIdx.x % ksplit) == rank) {
-        const int row = row0 + threadIdx.x;
-        float v = 0.f;
-        for (int q = 0; q < ksplit; ++q) v += *cluster.map_shared_rank(&partial[threadIdx.x], q);
-        if (row < N) {
-            if (bias) v += Dt<D>::to_f32(bias[row]);
-            y[row] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);
-        }
+template <typename D>
+cudaError_t launch_t(const void *x, const uint8_t *W, const float *absmax, const void *bias,
+                     void *y, int N, int K, int log2B, const CodeTable &tab, cudaStream_t stream) {
+    const int G = device_sm_count();
+    const int kpad = ((K + 31) / 32) * 32;
+    const size_t smem = kLut + (size_t)kWarps * STAGES * kSlot + kMaxRows * 4 + (size_t)kpad * 2;
+    static int smem_set = 0;  // largest dynamic shared memory size set so far
+    if ((int)smem > smem_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        smem_set = (int)smem;
     }
-    cluster.sync();  // keep every CTA's shared memory alive until all reads are done
+    gemv_kernel<D><<<G, kThreads, smem, stream>>>(
+        static_cast<const uint16_t *>(x), W, absmax, static_cast<const uint16_t *>(bias),
+        static_cast<uint16_t *>(y), N, K, log2B, tab);
+    return cudaGetLastError();
 }
 
 }  // namespace
+
+int64_t gemv_max_rows() { return (int64_t)device_sm_count() * kMaxRows; }
+int64_t gemv_max_k() { return kMaxK; }
 
 cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
                         void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
@@ -182,44 +253,10 @@ cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, co
     static const CodeTable nf4 = host_code_table(BNB4_NF4);
     static const CodeTable fp4 = host_code_table(BNB4_FP4);
     const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
-
-    const int sms = device_sm_count();
-    const int groups = (int)((N + kRowsPerCta - 1) / kRowsPerCta);
-    const int segs = (int)((K + kSeg - 1) / kSeg);
-    int ksplit = 1;
-    // enough CTAs to cover the GPU twice, and an x slice that fits 32 KB
-    while (ksplit < 8 && ksplit < segs &&
-           ((int64_t)groups * ksplit < 2 * sms || (K + ksplit - 1) / ksplit > kMaxKc))
-        ++ksplit;
-    // K-range per CTA in whole segments
-    const int segs_per = (segs + ksplit - 1) / ksplit;
-    ksplit = (segs + segs_per - 1) / segs_per;
-    int Kc = segs_per * kSeg;
-    if (Kc > K) Kc = (int)K;
-    if (Kc > kMaxKc) return cudaErrorInvalidValue;  // K > 8 * 8192: not reached by the API limits below
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(groups, ksplit, 1);
-    cfg.blockDim = dim3(kWarps * 32, 1, 1);
-    cfg.dynamicSmemBytes = (size_t)Kc * sizeof(float);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = ksplit;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-
-    const uint16_t *xp = static_cast<const uint16_t *>(x);
-    const uint16_t *bp = static_cast<const uint16_t *>(bias);
-    uint16_t *yp = static_cast<uint16_t *>(y);
     const int log2B = ilog2(blocksize);
     if (dt == BNB4_F16)
-        return cudaLaunchKernelEx(&cfg, gemv_kernel<F16>, xp, W, absmax, bp, yp, (int)N, (int)K,
-                                  log2B, Kc, tab);
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<BF16>, xp, W, absmax, bp, yp, (int)N, (int)K,
-                              log2B, Kc, tab);
+        return launch_t<F16>(x, W, absmax, bias, y, (int)N, (int)K, log2B, tab, stream);
+    return launch_t<BF16>(x, W, absmax, bias, y, (int)N, (int)K, log2B, tab, stream);
 }
 
 }  // namespace bnb4

@@ -20,7 +20,9 @@ cudaError_t launch_dequantize(const uint8_t *packed, const float *absmax, void *
                               int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
                               cudaStream_t stream);
 
-// M == 1, CUDA cores
+// M == 1, CUDA cores; handles N <= gemv_max_rows() and K <= gemv_max_k()
+int64_t gemv_max_rows();
+int64_t gemv_max_k();
 cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
                         void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
                         bnb4_dtype dt, cudaStream_t stream);

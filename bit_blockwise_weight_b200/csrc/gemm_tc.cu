@@ -14,8 +14,8 @@
 // accumulators (2 x 256 TMEM columns = all 512) that share one B operand:
 //   * warp 0, one thread: TMA loads of A (two 128 x 64 boxes per stage,
 //     128-byte swizzle) into a 3-stage ring;
-//   * warps 2-9: each thread decodes one 64-element weight run per stage
-//     (32 packed bytes + its block absmax) into a 128-byte row of the B tile
+//   * warps 2-9: each thread decodes one 64-element weight run per
+//     stage (32 packed bytes + its block absmax) into a 128-byte row of the B tile
 //     in the canonical 128-byte-swizzled layout: K-major rows for the forward,
 //     MN-major rows for the backward (so neither needs a transpose), then
 //     fences the writes to the async proxy and arrives on the stage barrier;
@@ -44,14 +44,17 @@ __device__ unsigned int g_device_error = 0;  // raised by a timed-out wait
 namespace {
 
 constexpr int BM = 256;           // two M=128 accumulators
-constexpr int BN = 256;           // output columns per tile
+constexpr int BN_MAX = 256;       // output columns per tile (256, or 224 to fill the SMs)
 constexpr int BK = 64;            // reduction per stage (one 128-byte swizzle row)
 constexpr int STAGES = 3;
 constexpr int A_HALF = 128 * BK * 2;             // 16 KB per 128-row box
 constexpr int A_STAGE = 2 * A_HALF;              // 32 KB
-constexpr int B_STAGE = BN * BK * 2;             // 32 KB
+constexpr int B_STAGE = BN_MAX * BK * 2;         // 32 KB
+constexpr int RED_CW = 64;                       // columns per reduction chunk (split K)
+constexpr int RED_PITCH = RED_CW + 4;            // fp32 staging row pitch
 constexpr int NUM_DQ_WARPS = 8;
 constexpr int THREADS = (2 + NUM_DQ_WARPS) * 32;  // 320
+constexpr int RUN_PARTS = NUM_DQ_WARPS / 8;       // threads per 64-weight run
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // ~1 s
 
 struct Smem {
@@ -190,6 +193,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes,
 }
 
 // Instruction descriptor for kind::f16: fp32 accumulate, M = 128, N = BN.
+template <int BN>
 __host__ __device__ constexpr uint32_t make_idesc(bool bf16, bool b_mn_major) {
     return (1u << 4)                              // D format: F32
            | ((bf16 ? 1u : 0u) << 7)              // A format
@@ -206,7 +210,46 @@ __device__ __forceinline__ uint32_t swz(uint32_t row_base, uint32_t row, uint32_
     return row_base + ((j ^ (row & 7u)) << 4);
 }
 
-template <typename D, bool BWD>
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t local_addr, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(remote)
+                 : "memory");
+    return v;
+}
+
+template <typename D>
+__device__ __forceinline__ void store_out(uint16_t *out, int64_t row, int n_out, int col,
+                                          const float *v, int cnt, const uint16_t *bias, bool add_bias) {
+    uint16_t *dst = out + row * n_out + col;
+    float w[16];
+    for (int e = 0; e < cnt; ++e) {
+        w[e] = v[e];
+        if (add_bias && bias && col + e < n_out) w[e] += Dt<D>::to_f32(bias[col + e]);
+    }
+    if (col + cnt <= n_out && cnt % 8 == 0 && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
+        for (int e = 0; e < cnt; e += 8) {
+            uint4 p;
+            p.x = Dt<D>::pack2(w[e], w[e + 1]);
+            p.y = Dt<D>::pack2(w[e + 2], w[e + 3]);
+            p.z = Dt<D>::pack2(w[e + 4], w[e + 5]);
+            p.w = Dt<D>::pack2(w[e + 6], w[e + 7]);
+            *reinterpret_cast<uint4 *>(dst + e) = p;
+        }
+    } else {
+        for (int e = 0; e < cnt && col + e < n_out; ++e) dst[e] = (uint16_t)(Dt<D>::pack2(w[e], 0.f) & 0xffffu);
+    }
+}
+
+template <typename D, bool BWD, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict__ W,
                const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
@@ -221,7 +264,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
     const int red = BWD ? N : K;    // reduction length
     const int c0 = blockIdx.x * BN;  // first output column of the tile
     const int m0 = blockIdx.y * BM;
-    const int iters = (red + BK - 1) / BK;
+    // split of the reduction over the CTAs of a cluster (gridDim.z of them)
+    const int C = gridDim.z, z = blockIdx.z;
+    const int iters_all = (red + BK - 1) / BK;
+    const int i_lo = (int)(((int64_t)iters_all * z) / C);
+    const int iters = (int)(((int64_t)iters_all * (z + 1)) / C) - i_lo;
     const int64_t row_bytes = K >> 1;
     const int nblk = K >> log2B;
 
@@ -255,8 +302,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
                 const int st = i % STAGES;
                 if (i >= STAGES && !mbar_wait(&s.empty[st], ((i / STAGES) - 1) & 1, abort)) break;
                 mbar_arrive_expect_tx(&s.full_a[st], A_STAGE);
-                tma_load_2d(&tmap_a, &s.full_a[st], s.a[st], i * BK, m0);
-                tma_load_2d(&tmap_a, &s.full_a[st], s.a[st] + A_HALF, i * BK, m0 + 128);
+                tma_load_2d(&tmap_a, &s.full_a[st], s.a[st], (i_lo + i) * BK, m0);
+                tma_load_2d(&tmap_a, &s.full_a[st], s.a[st] + A_HALF, (i_lo + i) * BK, m0 + 128);
             }
             // do not leave while a load may still be landing in this CTA's memory
             for (int i = (iters > STAGES ? iters - STAGES : 0); i < iters; ++i)
@@ -265,7 +312,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc(std::is_same<D, BF16>::value, BWD);
+            constexpr uint32_t idesc = make_idesc<BN>(std::is_same<D, BF16>::value, BWD);
             bool ok = true;
             for (int i = 0; i < iters && ok; ++i) {
                 const int st = i % STAGES;
@@ -293,31 +340,40 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
             if (ok) tc_commit(&s.tmem_full);
         }
     } else {
-        // -------------------------------------- weight dequant (warps 2..9)
-        const int t = threadIdx.x - 64;  // 0..255: one 64-element weight run per stage
+        // ---------------------------------------- weight dequant warps
+        // 256 runs of 64 weights per stage; RUN_PARTS threads share a run, each
+        // decoding 32 / RUN_PARTS packed bytes into 8 / RUN_PARTS of its chunks
+        const int part = (threadIdx.x - 64) >> 8;
+        const int t = (threadIdx.x - 64) & 255;
+        constexpr int WORDS = 8 / RUN_PARTS;
         const uint32_t my_code = __float_as_uint(tab.v[lane & 15]);
         // run geometry: forward row t of the tile (output column c0 + t) over the
         // stage's 64 reduction indices; backward reduction row (t & 63) of the
         // stage over output columns c0 + 64 (t >> 6) ... + 63
         auto src = [&](int i, int &wrow, int &kcol) {
             if (BWD) {
-                wrow = i * BK + (t & 63);
+                wrow = (i_lo + i) * BK + (t & 63);
                 kcol = c0 + 64 * (t >> 6);
             } else {
-                wrow = c0 + t;
-                kcol = i * BK;
+                wrow = t < BN ? c0 + t : N;  // threads past the tile width decode nothing
+                kcol = (i_lo + i) * BK;
             }
         };
-        auto fetch = [&](int i, uint4 &w0, uint4 &w1, float &a) {
+        auto fetch = [&](int i, uint32_t (&w)[WORDS], float &a) {
             int wrow, kcol;
             src(i, wrow, kcol);
             if (wrow < N && kcol < K) {
-                const uint4 *p = reinterpret_cast<const uint4 *>(W + (int64_t)wrow * row_bytes + (kcol >> 1));
-                w0 = __ldg(p);
-                w1 = __ldg(p + 1);
+                const uint4 *p = reinterpret_cast<const uint4 *>(W + (int64_t)wrow * row_bytes + (kcol >> 1)) +
+                                 part * (WORDS / 4);
+#pragma unroll
+                for (int q = 0; q < WORDS / 4; ++q) {
+                    const uint4 v = __ldg(p + q);
+                    w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+                }
                 a = __ldg(absmax + (int64_t)wrow * nblk + (kcol >> log2B));
             } else {
-                w0 = w1 = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int q = 0; q < WORDS; ++q) w[q] = 0u;
                 a = 0.0f;  // zero weights past the edges
             }
         };
@@ -331,69 +387,121 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
             row_base = (t >> 3) * 1024 + (t & 7) * 128;
             row_sw = t;
         }
-        uint4 w0, w1, n0, n1;
+        uint32_t w[WORDS], nw[WORDS];
         float a, na;
-        if (iters > 0) fetch(0, w0, w1, a);
+        if (iters > 0) fetch(0, w, a);
         for (int i = 0; i < iters; ++i) {
             const int st = i % STAGES;
-            if (i + 1 < iters) fetch(i + 1, n0, n1, na);
+            if (i + 1 < iters) fetch(i + 1, nw, na);
             if (i >= STAGES && !mbar_wait(&s.empty[st], ((i / STAGES) - 1) & 1, abort)) break;
             uint8_t *bt = s.b[st];
-            const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = weights 8j .. 8j+7 = bytes 4j..4j+3
+            for (int jj = 0; jj < WORDS; ++jj) {  // chunk j = weights 8j .. 8j+7 = bytes 4j..4j+3
+                const int j = WORDS * part + jj;
                 uint32_t o[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const uint32_t byte_sh = 8 * h;  // byte h of word j
-                    const float ch = __uint_as_float(shfl_idx(my_code, w[j] >> (byte_sh + 4)));
-                    const float cl = __uint_as_float(shfl_idx(my_code, w[j] >> byte_sh));
+                    const float ch = __uint_as_float(shfl_idx(my_code, w[jj] >> (byte_sh + 4)));
+                    const float cl = __uint_as_float(shfl_idx(my_code, w[jj] >> byte_sh));
                     o[h] = Dt<D>::pack2(__fmul_rn(ch, a), __fmul_rn(cl, a));
                 }
-                *reinterpret_cast<uint4 *>(bt + swz(row_base, row_sw, j)) = make_uint4(o[0], o[1], o[2], o[3]);
+                if (BWD || t < BN)
+                    *reinterpret_cast<uint4 *>(bt + swz(row_base, row_sw, j)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async();
             mbar_arrive(&s.full_b[st]);
-            w0 = n0;
-            w1 = n1;
+#pragma unroll
+            for (int q = 0; q < WORDS; ++q) w[q] = nw[q];
             a = na;
         }
 
-        // ------------------------------------------------------- epilogue
-        __syncwarp();
-        if (mbar_wait(&s.tmem_full, 0, abort)) {
+        // ------------------------------------------------ direct epilogue
+        if (C == 1) {
             __syncwarp();
-            tc_fence_after();
-            const int q = warp & 3;              // TMEM lane quadrant this warp may read
-            const int mt = (warp - 2) >> 2;      // accumulator: warps 2-5 -> 0, 6-9 -> 1
-            const int row = m0 + mt * 128 + q * 32 + lane;
-            const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
+            if (mbar_wait(&s.tmem_full, 0, abort)) {
+                __syncwarp();
+                tc_fence_after();
+                // warp 2 + ew: TMEM lane quadrant warp & 3 (the one it may read),
+                // accumulator (ew >> 2) & 1, column part ew >> 3
+                const int ew = warp - 2;
+                const int q = warp & 3;
+                const int mt = (ew >> 2) & 1;
+                const int row = m0 + mt * 128 + q * 32 + lane;
+                const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
+                const int cbeg = (ew >> 3) * (BN / RUN_PARTS);
 #pragma unroll 1
-            for (int cc = 0; cc < BN; cc += 16) {
-                uint32_t r[16];
-                tmem_ld16(tbase + cc, r);
-                tmem_ld_wait();
-                const int col = c0 + cc;
-                if (row < M && col < n_out) {
-                    float v[16];
+                for (int cc = cbeg; cc < cbeg + BN / RUN_PARTS; cc += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tbase + cc, r);
+                    tmem_ld_wait();
+                    const int col = c0 + cc;
+                    if (row < M && col < n_out) {
+                        float v[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        v[e] = __uint_as_float(r[e]);
-                        if (!BWD && bias && col + e < n_out) v[e] += Dt<D>::to_f32(bias[col + e]);
-                    }
-                    uint16_t *dst = out + (int64_t)row * n_out + col;
-                    if (col + 16 <= n_out && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
-                        uint32_t p[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) p[e] = Dt<D>::pack2(v[2 * e], v[2 * e + 1]);
-                        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(p[0], p[1], p[2], p[3]);
-                        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(p[4], p[5], p[6], p[7]);
-                    } else {
-                        for (int e = 0; e < 16 && col + e < n_out; ++e)
-                            dst[e] = (uint16_t)(Dt<D>::pack2(v[e], 0.f) & 0xffffu);
+                        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]);
+                        store_out<D>(out, row, n_out, col, v, 16, bias, !BWD);
                     }
                 }
             }
+        }
+    }
+
+    // ------------------- split reduction: add the cluster's partial tiles
+    // Every thread of every CTA of the cluster passes the same cluster
+    // barriers, whatever happened before, so none can be left waiting.
+    if (C > 1) {
+        __syncwarp();
+        bool have = false;
+        if (warp >= 2) {
+            have = __all_sync(FULL, mbar_wait(&s.tmem_full, 0, abort));
+            if (have) tc_fence_after();
+        }
+        // the A ring is free once the last MMA has completed: fp32 staging of
+        // one 256 x 64 chunk of this CTA's partial tile
+        float *stg = reinterpret_cast<float *>(&s.a[0][0]);
+        const uint32_t stg_addr = smem_u32(stg);
+        const int rows_per = BM / C;
+#pragma unroll 1
+        for (int cb = 0; cb < BN; cb += RED_CW) {
+            if (warp >= 2 && have) {
+                const int ew = warp - 2;
+                const int q = warp & 3, mt = (ew >> 2) & 1;
+                const int lrow = mt * 128 + q * 32 + lane;
+                const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
+                const int cbeg = (ew >> 3) * (RED_CW / RUN_PARTS);
+#pragma unroll
+                for (int cc = cbeg; cc < cbeg + RED_CW / RUN_PARTS; cc += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(tbase + cb + cc, r);
+                    tmem_ld_wait();
+                    float4 *d = reinterpret_cast<float4 *>(stg + lrow * RED_PITCH + cc);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        d[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                           __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                }
+            }
+            cluster_sync_all();
+            if (warp >= 2) {
+                const int e0 = threadIdx.x - 64;
+                for (int v = e0; v < rows_per * (RED_CW / 4); v += NUM_DQ_WARPS * 32) {
+                    const int lr = z * rows_per + v / (RED_CW / 4);
+                    const int c4 = (v % (RED_CW / 4)) * 4;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const uint32_t la = stg_addr + (uint32_t)(lr * RED_PITCH + c4) * 4;
+                    for (int q2 = 0; q2 < C; ++q2) {
+                        const float4 p = ld_dsmem_f4(la, (uint32_t)q2);
+                        acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+                    }
+                    const int row = m0 + lr, col = c0 + cb + c4;
+                    if (row < M && col < n_out) {
+                        const float vv[4] = {acc.x, acc.y, acc.z, acc.w};
+                        store_out<D>(out, row, n_out, col, vv, 4, bias, !BWD);
+                    }
+                }
+            }
+            cluster_sync_all();
         }
     }
 
@@ -418,6 +526,42 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
+template <typename D, bool BWD, int BN>
+cudaError_t launch_bn(const CUtensorMap &map, const uint8_t *W, const float *absmax,
+                      const void *bias, void *out, int M, int N, int K, int log2B,
+                      const CodeTable &tab, int C, cudaStream_t stream) {
+    const size_t smem = sizeof(Smem) + 1024;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<D, BWD, BN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int n_out = BWD ? K : N;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((n_out + BN - 1) / BN, (M + BM - 1) / BM, C);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = C;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<D, BWD, BN>, map, W, absmax,
+                              static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(out), M,
+                              N, K, log2B, tab);
+}
+
+// fraction of the SM slots that the last wave of `tiles` one-SM CTAs leaves busy
+double wave_eff(long tiles, int sms) {
+    const long waves = (tiles + sms - 1) / sms;
+    return (double)tiles / (double)(waves * sms);
+}
+
 template <typename D, bool BWD>
 cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const void *bias,
                      void *out, int M, int N, int K, int log2B, const CodeTable &tab,
@@ -440,19 +584,24 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-    const size_t smem = sizeof(Smem) + 1024;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<D, BWD>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
+    const int sms = device_sm_count();
+    const long mt = (M + BM - 1) / BM;
+    // tile width: 224 when it fills the SMs better (forward only; the backward's
+    // MN-major weight tile is built from 64-column atoms)
+    int bn = 256;
+    if (!BWD && wave_eff(mt * ((n_out + 223) / 224), sms) > wave_eff(mt * ((n_out + 255) / 256), sms) + 0.02)
+        bn = 224;
+    const long tiles = mt * ((n_out + bn - 1) / bn);
+    // split the reduction over a cluster when the tiles alone leave SMs idle
+    // and every CTA keeps at least 16 stages
+    const int iters = (red + BK - 1) / BK;
+    int C = 1;
+    while (C < 8 && tiles * (2 * C) <= sms && iters / (2 * C) >= 16) C *= 2;
+    if constexpr (!BWD) {
+        if (bn == 224)
+            return launch_bn<D, BWD, 224>(map, W, absmax, bias, out, M, N, K, log2B, tab, C, stream);
     }
-    dim3 grid((n_out + BN - 1) / BN, (M + BM - 1) / BM);
-    gemm_tc_kernel<D, BWD><<<grid, THREADS, smem, stream>>>(
-        map, W, absmax, static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(out), M, N,
-        K, log2B, tab);
-    return cudaGetLastError();
+    return launch_bn<D, BWD, 256>(map, W, absmax, bias, out, M, N, K, log2B, tab, C, stream);
 }
 
 }  // namespace

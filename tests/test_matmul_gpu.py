@@ -118,8 +118,11 @@ def _ref_backward(Wt, dYs, dt, M, entries=None):
 @pytest.mark.parametrize("q", ["nf4", "fp4"])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 @pytest.mark.parametrize("M,N,K,B", [(17, 256, 256, 64), (100, 320, 512, 64), (256, 512, 1024, 128),
-                                     (300, 96, 256, 256), (257, 264, 704, 64)])
+                                     (300, 96, 256, 256), (257, 264, 704, 64), (300, 256, 4096, 64),
+                                     (300, 33152, 256, 64)])
 def test_gemm_large_m(q, dt, M, N, K, B):
+    """Includes a reduction split over a cluster (K=4096, two tiles) and a width
+    (N = 148 * 224) where 224-column tiles fill the SMs."""
     Wt = Weight(N, K, B, q, seed=M)
     Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
     bs = synthetic.storage_numpy(synthetic.bias(N, seed=2, dtype=dt)) if M % 2 == 0 else None
@@ -133,8 +136,10 @@ def test_gemm_large_m(q, dt, M, N, K, B):
 @pytest.mark.parametrize("q", ["nf4", "fp4"])
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 @pytest.mark.parametrize("M,N,K,B", [(1, 256, 256, 64), (17, 256, 512, 64), (256, 200, 256, 64),
-                                     (300, 320, 768, 256), (64, 1024, 1280, 128)])
+                                     (300, 320, 768, 256), (64, 1024, 1280, 128),
+                                     (64, 8192, 256, 64), (300, 4096, 512, 128)])
 def test_gemm_backward(q, dt, M, N, K, B):
+    """Includes reductions long enough to be split over a thread-block cluster."""
     Wt = Weight(N, K, B, q, seed=N)
     dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3, dtype=dt)).reshape(-1)
     dX = bnb4.gemm_4bit_backward(to_dev(dYs, dt).view(M, N), Wt.dp, Wt.da, K, B, q)

@@ -454,6 +454,49 @@ def run_reference(args):
                     "d2h_bytes_per_step": 0}}
 
 
+PROFILE_CASES = {
+    # name: what runs (inputs above L2 size, a few hundred MB on the device at most)
+    "quantize": "quantize_4bit, 2^26 bf16 elements, NF4, B=64",
+    "dequantize": "dequantize_4bit, 2^26 elements to bf16, NF4, B=64",
+    "gemv": "gemv_4bit + bias, K=4096, N=14336, NF4 B=64, bf16",
+    "gemm_small": "gemm_4bit M=16, K=8192, N=28672, NF4 B=64, bf16",
+    "gemm_tc": "gemm_4bit M=512, K=4096, N=14336, NF4 B=64, bf16",
+    "gemm_tc_backward": "gemm_4bit_backward M=512, K=4096, N=14336, NF4 B=64, bf16",
+}
+
+
+def profile_case(name):
+    """One launch of one kernel on a small case, for an ncu capture (no timing, no JSON line).
+
+    Setup launches (input draws, weight quantization) come first; the kernel of
+    interest is the last launch of its kind."""
+    import bit_blockwise_weight_b200 as bnb4
+    from bit_blockwise_weight_b200 import synthetic
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    d = str(dev)
+    if name in ("quantize", "dequantize"):
+        x = synthetic.roundtrip_tensor(1 << 26, 0, "bf16", device=d)
+        p, a = bnb4.quantize_4bit(x, BLOCK, "nf4")
+        if name == "dequantize":
+            bnb4.dequantize_4bit(p, a, x.numel(), BLOCK, "nf4", dtype=torch.bfloat16)
+    else:
+        K, N, M = {"gemv": (4096, 14336, 1), "gemm_small": (8192, 28672, 16),
+                   "gemm_tc": (4096, 14336, 512), "gemm_tc_backward": (4096, 14336, 512)}[name]
+        w = synthetic.normal((N * K,), 0, 0.02, "f32", device=d)
+        p, a = bnb4.quantize_4bit(w, BLOCK, "nf4")
+        del w
+        if name == "gemv":
+            bnb4.gemv_4bit(synthetic.normal((K,), 1, 1.0, "bf16", device=d), p, a, N, K,
+                           synthetic.normal((N,), 2, 1.0, "bf16", device=d))
+        elif name == "gemm_tc_backward":
+            bnb4.gemm_4bit_backward(synthetic.normal((M, N), 3, 1.0, "bf16", device=d), p, a, K)
+        else:
+            bnb4.gemm_4bit(synthetic.normal((M, K), 1, 1.0, "bf16", device=d), p, a, N)
+    torch.cuda.synchronize(dev)
+    print(f"profile case {name}: {PROFILE_CASES[name]}")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -462,7 +505,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run one launch of one kernel on a small case for an ncu capture "
+                         "(prints no bench line)")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         args.warmup = 3
 

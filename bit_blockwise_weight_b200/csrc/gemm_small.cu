@@ -89,7 +89,7 @@ template <typename D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_small_kernel(const uint16_t *__restrict__ X, const uint8_t *__restrict__ W,
                   const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-                  uint16_t *__restrict__ Y, int M, int N, int K, int log2B, CodeTable tab) {
+                  uint16_t *__restrict__ Y, int M, int N, int K, int log2B, const __grid_constant__ CodeTable tab) {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem);                 // 256 x 32 words
     float *sum = reinterpret_cast<float *>(smem + 256 * 32 * 4);        // [kMaxTiles*16][16]

@@ -10,21 +10,31 @@
 //   forward   D[M, N] = A[M, K] . W[N, K]^T   (A = X,  reduction over K)
 //   backward  D[M, K] = A[M, N] . W[N, K]     (A = dY, reduction over N)
 //
-// One CTA computes a 256 x 256 output tile as two M=128 tcgen05.mma
-// accumulators (2 x 256 TMEM columns = all 512) that share one B operand:
+// One CTA computes a 256 x BN output tile (BN = 256, or 224 when that fills
+// the SMs better) as two M=128 tcgen05.mma accumulators (2 x BN TMEM columns)
+// that share one B operand:
 //   * warp 0, one thread: TMA loads of A (two 128 x 64 boxes per stage,
-//     128-byte swizzle) into a 3-stage ring;
-//   * warps 2-9: each thread decodes one 64-element weight run per
-//     stage (32 packed bytes + its block absmax) into a 128-byte row of the B tile
-//     in the canonical 128-byte-swizzled layout: K-major rows for the forward,
-//     MN-major rows for the backward (so neither needs a transpose), then
-//     fences the writes to the async proxy and arrives on the stage barrier;
-//   * warp 1, one thread: waits for both halves of a stage, issues 2 x 4
-//     tcgen05.mma (K = 16 each) and commits the stage back to the producers;
+//     128-byte swizzle) into a 3-slot ring;
+//   * warp 10: TMA loads of the stage's packed weight tile (BN rows x 32 bytes,
+//     32-byte swizzle, forward; 64 rows x 128 bytes, 128-byte swizzle,
+//     backward) and of the matching absmax tile (16 bytes per weight row) into
+//     a 4-slot ring.  When the absmax row pitch is not a multiple of 16 bytes
+//     the warp gathers the absmax values with ordinary loads instead;
+//   * warps 2-9: each thread reads one 64-element weight run (32 packed bytes
+//     + its block absmax) from the ring, decodes it and writes one 128-byte row
+//     of the B tile in the canonical 128-byte-swizzled layout: K-major rows for
+//     the forward, MN-major rows for the backward (so neither needs a
+//     transpose), fences the writes to the async proxy and arrives on the stage
+//     barrier of a 2-slot B ring;
+//   * warp 1, one thread: waits for A and B of a stage, issues 2 x 4
+//     tcgen05.mma (K = 16 each) and commits the slots back to the producers;
 //   * after the last stage warps 2-9 read the accumulators (tcgen05.ld), add
 //     the bias in fp32, round once and store.
 // Each decoded weight is RN_dtype(fp32(code * absmax)), the exact value the
 // dequantize kernel produces, so the MMA consumes the dequantized weight.
+// Packed-weight bytes that the tensor map clips (rows past N, bytes past K/2)
+// arrive as zeros; the absmax tile is clipped the same way, so rows past N
+// decode to +-0, and columns past K meet zero-filled A columns.
 //
 // Every mbarrier wait is bounded (about one second of %globaltimer); a wait
 // that runs out raises the library's device error word, makes the CTA skip
@@ -32,6 +42,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <type_traits>
 
 #include "common.cuh"
@@ -46,27 +57,35 @@ namespace {
 constexpr int BM = 256;           // two M=128 accumulators
 constexpr int BN_MAX = 256;       // output columns per tile (256, or 224 to fill the SMs)
 constexpr int BK = 64;            // reduction per stage (one 128-byte swizzle row)
-constexpr int STAGES = 3;
+constexpr int A_STAGES = 3;
+constexpr int B_STAGES = 2;
+constexpr int W_STAGES = 4;
 constexpr int A_HALF = 128 * BK * 2;             // 16 KB per 128-row box
 constexpr int A_STAGE = 2 * A_HALF;              // 32 KB
 constexpr int B_STAGE = BN_MAX * BK * 2;         // 32 KB
+constexpr int W_SLOT = BN_MAX * BK / 2;          // 8 KB of packed weights per stage
+constexpr int AMX_SLOT = BN_MAX * 4;             // 4 floats per weight row
 constexpr int RED_CW = 64;                       // columns per reduction chunk (split K)
 constexpr int RED_PITCH = RED_CW + 4;            // fp32 staging row pitch
 constexpr int NUM_DQ_WARPS = 8;
-constexpr int THREADS = (2 + NUM_DQ_WARPS) * 32;  // 320
-constexpr int RUN_PARTS = NUM_DQ_WARPS / 8;       // threads per 64-weight run
+constexpr int W_WARP = 2 + NUM_DQ_WARPS;          // weight-tile producer
+constexpr int THREADS = (3 + NUM_DQ_WARPS) * 32;  // 352
 constexpr uint64_t kWaitLimitNs = 1000000000ull;  // ~1 s
 
 struct Smem {
-    uint8_t a[STAGES][A_STAGE];   // 1024-byte aligned (swizzle atoms)
-    uint8_t b[STAGES][B_STAGE];
-    uint64_t full_a[STAGES];
-    uint64_t full_b[STAGES];
-    uint64_t empty[STAGES];
+    uint8_t a[A_STAGES][A_STAGE];   // 1024-byte aligned (swizzle atoms)
+    uint8_t b[B_STAGES][B_STAGE];
+    uint8_t w[W_STAGES][W_SLOT];
+    float amx[W_STAGES][AMX_SLOT];
+    uint64_t full_a[A_STAGES], empty_a[A_STAGES];
+    uint64_t full_b[B_STAGES], empty_b[B_STAGES];
+    uint64_t full_w[W_STAGES], empty_w[W_STAGES];
     uint64_t tmem_full;
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory plan");
+static_assert(BM * RED_PITCH * 4 <= A_STAGES * A_STAGE, "split-K staging fits in the A ring");
 
 // ------------------------------------------------------------------ PTX
 
@@ -226,17 +245,19 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t local_addr, uint32_t rank
     return v;
 }
 
-template <typename D>
+template <typename D, int CNT>
 __device__ __forceinline__ void store_out(uint16_t *out, int64_t row, int n_out, int col,
-                                          const float *v, int cnt, const uint16_t *bias, bool add_bias) {
+                                          const float *v, const uint16_t *bias, bool add_bias) {
     uint16_t *dst = out + row * n_out + col;
-    float w[16];
-    for (int e = 0; e < cnt; ++e) {
+    float w[CNT];
+#pragma unroll
+    for (int e = 0; e < CNT; ++e) {
         w[e] = v[e];
         if (add_bias && bias && col + e < n_out) w[e] += Dt<D>::to_f32(bias[col + e]);
     }
-    if (col + cnt <= n_out && cnt % 8 == 0 && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0)) {
-        for (int e = 0; e < cnt; e += 8) {
+    if (col + CNT <= n_out && ((reinterpret_cast<uintptr_t>(dst) & 15) == 0) && CNT % 8 == 0) {
+#pragma unroll
+        for (int e = 0; e < CNT; e += 8) {
             uint4 p;
             p.x = Dt<D>::pack2(w[e], w[e + 1]);
             p.y = Dt<D>::pack2(w[e + 2], w[e + 3]);
@@ -244,16 +265,35 @@ __device__ __forceinline__ void store_out(uint16_t *out, int64_t row, int n_out,
             p.w = Dt<D>::pack2(w[e + 6], w[e + 7]);
             *reinterpret_cast<uint4 *>(dst + e) = p;
         }
+    } else if (col + CNT <= n_out && ((reinterpret_cast<uintptr_t>(dst) & 7) == 0) && CNT % 4 == 0) {
+#pragma unroll
+        for (int e = 0; e < CNT; e += 4)
+            *reinterpret_cast<uint2 *>(dst + e) =
+                make_uint2(Dt<D>::pack2(w[e], w[e + 1]), Dt<D>::pack2(w[e + 2], w[e + 3]));
     } else {
-        for (int e = 0; e < cnt && col + e < n_out; ++e) dst[e] = (uint16_t)(Dt<D>::pack2(w[e], 0.f) & 0xffffu);
+#pragma unroll
+        for (int e = 0; e < CNT; ++e)
+            if (col + e < n_out) dst[e] = (uint16_t)(Dt<D>::pack2(w[e], 0.f) & 0xffffu);
     }
+}
+
+// Bounded wait used before a CTA exits: lets loads still in flight land in its
+// shared memory even when the CTA is aborting.
+__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) {
+            atomicAdd(&g_device_error, 1u);
+            return;
+        }
 }
 
 template <typename D, bool BWD, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict__ W,
-               const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-               uint16_t *__restrict__ out, int M, int N, int K, int log2B, CodeTable tab) {
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
+               const __grid_constant__ CUtensorMap tmap_amx, const float *__restrict__ absmax,
+               const uint16_t *__restrict__ bias, uint16_t *__restrict__ out, int M, int N, int K,
+               int log2B, int amx_tma, const __grid_constant__ CodeTable tab) {
     extern __shared__ uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~(uintptr_t)1023);
@@ -269,14 +309,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
     const int iters_all = (red + BK - 1) / BK;
     const int i_lo = (int)(((int64_t)iters_all * z) / C);
     const int iters = (int)(((int64_t)iters_all * (z + 1)) / C) - i_lo;
-    const int64_t row_bytes = K >> 1;
     const int nblk = K >> log2B;
+    // first absmax column of the 16-byte box that holds a stage's scales
+    // (backward: fixed per tile; forward: per stage)
+    const int bwd_x0 = (c0 >> log2B) & ~3;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGES; ++i) {
+        for (int i = 0; i < A_STAGES; ++i) {
             mbar_init(&s.full_a[i], 1);
+            mbar_init(&s.empty_a[i], 1);
+        }
+        for (int i = 0; i < B_STAGES; ++i) {
             mbar_init(&s.full_b[i], NUM_DQ_WARPS * 32);
-            mbar_init(&s.empty[i], 1);
+            mbar_init(&s.empty_b[i], 1);
+        }
+        for (int i = 0; i < W_STAGES; ++i) {
+            mbar_init(&s.full_w[i], 32);
+            mbar_init(&s.empty_w[i], NUM_DQ_WARPS * 32);
         }
         mbar_init(&s.tmem_full, 1);
         s.abort = 0;
@@ -298,30 +347,89 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a))
                          : "memory");
+            int issued = 0;
             for (int i = 0; i < iters; ++i) {
-                const int st = i % STAGES;
-                if (i >= STAGES && !mbar_wait(&s.empty[st], ((i / STAGES) - 1) & 1, abort)) break;
+                const int st = i % A_STAGES;
+                if (i >= A_STAGES && !mbar_wait(&s.empty_a[st], ((i / A_STAGES) - 1) & 1, abort)) break;
                 mbar_arrive_expect_tx(&s.full_a[st], A_STAGE);
                 tma_load_2d(&tmap_a, &s.full_a[st], s.a[st], (i_lo + i) * BK, m0);
                 tma_load_2d(&tmap_a, &s.full_a[st], s.a[st] + A_HALF, (i_lo + i) * BK, m0 + 128);
+                issued = i + 1;
             }
             // do not leave while a load may still be landing in this CTA's memory
-            for (int i = (iters > STAGES ? iters - STAGES : 0); i < iters; ++i)
-                if (!mbar_wait(&s.full_a[i % STAGES], (i / STAGES) & 1, abort)) break;
+            for (int i = (issued > A_STAGES ? issued - A_STAGES : 0); i < issued; ++i)
+                mbar_drain(&s.full_a[i % A_STAGES], (i / A_STAGES) & 1);
         }
+    } else if (warp == W_WARP) {
+        // ---------------------------------- TMA producer (packed weights, absmax)
+        constexpr int W_ROWS = BWD ? BK : BN;  // weight rows per stage
+        constexpr uint32_t W_BYTES = W_ROWS * (BWD ? BN_MAX / 2 : BK / 2);
+        const uint32_t tx = W_BYTES + (amx_tma ? W_ROWS * 16u : 0u);
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w))
+                         : "memory");
+            if (amx_tma)
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_amx))
+                             : "memory");
+        }
+        int issued = 0;
+        for (int i = 0; i < iters; ++i) {
+            const int st = i % W_STAGES;
+            bool ok = true;
+            if (i >= W_STAGES) ok = mbar_wait(&s.empty_w[st], ((i / W_STAGES) - 1) & 1, abort);
+            if (!__all_sync(FULL, ok)) break;
+            const int it = i_lo + i;
+            if (!amx_tma) {
+                // gather the stage's scales into the same [row][4] layout the
+                // tensor map would produce
+                float *dst = s.amx[st];
+                for (int p = lane; p < 256; p += 32) {
+                    int row, blk, idx;
+                    if (BWD) {
+                        row = it * BK + (p & 63);
+                        blk = (c0 + 64 * (p >> 6)) >> log2B;
+                        idx = blk - bwd_x0;
+                        if (p < 64 * 4) dst[(p & 63) * 4 + idx] =
+                            (row < N && blk < nblk) ? __ldg(absmax + (int64_t)row * nblk + blk) : 0.0f;
+                    } else {
+                        row = c0 + p;
+                        blk = (it * BK) >> log2B;
+                        idx = blk & 3;
+                        if (p < BN) dst[p * 4 + idx] = row < N ? __ldg(absmax + (int64_t)row * nblk + blk) : 0.0f;
+                    }
+                }
+            }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&s.full_w[st], tx);
+                if (BWD) {
+                    tma_load_2d(&tmap_w, &s.full_w[st], s.w[st], c0 >> 1, it * BK);
+                    if (amx_tma) tma_load_2d(&tmap_amx, &s.full_w[st], s.amx[st], bwd_x0, it * BK);
+                } else {
+                    tma_load_2d(&tmap_w, &s.full_w[st], s.w[st], it * (BK / 2), c0);
+                    if (amx_tma)
+                        tma_load_2d(&tmap_amx, &s.full_w[st], s.amx[st], ((it * BK) >> log2B) & ~3, c0);
+                }
+            } else {
+                mbar_arrive(&s.full_w[st]);
+            }
+            issued = i + 1;
+        }
+        if (lane == 0)
+            for (int i = (issued > W_STAGES ? issued - W_STAGES : 0); i < issued; ++i)
+                mbar_drain(&s.full_w[i % W_STAGES], (i / W_STAGES) & 1);
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc<BN>(std::is_same<D, BF16>::value, BWD);
             bool ok = true;
             for (int i = 0; i < iters && ok; ++i) {
-                const int st = i % STAGES;
-                const uint32_t par = (i / STAGES) & 1;
-                ok = mbar_wait(&s.full_a[st], par, abort) && mbar_wait(&s.full_b[st], par, abort);
+                const int sa = i % A_STAGES, sb = i % B_STAGES;
+                ok = mbar_wait(&s.full_a[sa], (i / A_STAGES) & 1, abort) &&
+                     mbar_wait(&s.full_b[sb], (i / B_STAGES) & 1, abort);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t a_base = smem_u32(s.a[st]);
-                const uint32_t b_base = smem_u32(s.b[st]);
+                const uint32_t a_base = smem_u32(s.a[sa]);
+                const uint32_t b_base = smem_u32(s.b[sb]);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     // B: K-major rows of 128 B (forward), or MN-major with the four
@@ -335,48 +443,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
                         tc_mma(tmem + mt * BN, adesc, bdesc, idesc, (i > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                tc_commit(&s.empty[st]);  // stage free once these MMAs have read it
+                tc_commit(&s.empty_a[sa]);  // slots free once these MMAs have read them
+                tc_commit(&s.empty_b[sb]);
             }
             if (ok) tc_commit(&s.tmem_full);
         }
     } else {
         // ---------------------------------------- weight dequant warps
-        // 256 runs of 64 weights per stage; RUN_PARTS threads share a run, each
-        // decoding 32 / RUN_PARTS packed bytes into 8 / RUN_PARTS of its chunks
-        const int part = (threadIdx.x - 64) >> 8;
-        const int t = (threadIdx.x - 64) & 255;
-        constexpr int WORDS = 8 / RUN_PARTS;
+        // 256 runs of 64 weights per stage, one per thread
+        const int t = threadIdx.x - 64;
         const uint32_t my_code = __float_as_uint(tab.v[lane & 15]);
-        // run geometry: forward row t of the tile (output column c0 + t) over the
-        // stage's 64 reduction indices; backward reduction row (t & 63) of the
-        // stage over output columns c0 + 64 (t >> 6) ... + 63
-        auto src = [&](int i, int &wrow, int &kcol) {
-            if (BWD) {
-                wrow = (i_lo + i) * BK + (t & 63);
-                kcol = c0 + 64 * (t >> 6);
-            } else {
-                wrow = t < BN ? c0 + t : N;  // threads past the tile width decode nothing
-                kcol = (i_lo + i) * BK;
-            }
-        };
-        auto fetch = [&](int i, uint32_t (&w)[WORDS], float &a) {
-            int wrow, kcol;
-            src(i, wrow, kcol);
-            if (wrow < N && kcol < K) {
-                const uint4 *p = reinterpret_cast<const uint4 *>(W + (int64_t)wrow * row_bytes + (kcol >> 1)) +
-                                 part * (WORDS / 4);
-#pragma unroll
-                for (int q = 0; q < WORDS / 4; ++q) {
-                    const uint4 v = __ldg(p + q);
-                    w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
-                }
-                a = __ldg(absmax + (int64_t)wrow * nblk + (kcol >> log2B));
-            } else {
-#pragma unroll
-                for (int q = 0; q < WORDS; ++q) w[q] = 0u;
-                a = 0.0f;  // zero weights past the edges
-            }
-        };
+        // forward: row t of the tile (output column c0 + t) over the stage's 64
+        // reduction indices; backward: reduction row (t & 63) of the stage over
+        // output columns c0 + 64 (t >> 6) ... + 63
+        const bool active = BWD || t < BN;
+        // source of the run in a weight slot, as two swizzled 16-byte chunks
+        uint32_t src0, src1;
+        if (BWD) {
+            const uint32_t r = t & 63, g = t >> 6;
+            src0 = r * 128 + (((2 * g) ^ (r & 7)) << 4);
+            src1 = r * 128 + (((2 * g + 1) ^ (r & 7)) << 4);
+        } else {
+            src0 = t * 32 + ((0u ^ ((t >> 2) & 1)) << 4);
+            src1 = t * 32 + ((1u ^ ((t >> 2) & 1)) << 4);
+        }
+        // absmax slot index: [row][4], the column inside the 16-byte box
+        const int amx_row = BWD ? (t & 63) : t;
+        const int bwd_idx = ((c0 + 64 * (t >> 6)) >> log2B) - bwd_x0;
         // destination row of this run in the B tile
         uint32_t row_base, row_sw;
         if (BWD) {
@@ -387,32 +480,49 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
             row_base = (t >> 3) * 1024 + (t & 7) * 128;
             row_sw = t;
         }
-        uint32_t w[WORDS], nw[WORDS];
-        float a, na;
-        if (iters > 0) fetch(0, w, a);
-        for (int i = 0; i < iters; ++i) {
-            const int st = i % STAGES;
-            if (i + 1 < iters) fetch(i + 1, nw, na);
-            if (i >= STAGES && !mbar_wait(&s.empty[st], ((i / STAGES) - 1) & 1, abort)) break;
-            uint8_t *bt = s.b[st];
+        auto load = [&](int i, uint32_t (&w)[8], float &a) -> bool {
+            const int ws = i % W_STAGES;
+            if (!mbar_wait(&s.full_w[ws], (i / W_STAGES) & 1, abort)) return false;
+            if (active) {
+                const uint4 v0 = *reinterpret_cast<const uint4 *>(s.w[ws] + src0);
+                const uint4 v1 = *reinterpret_cast<const uint4 *>(s.w[ws] + src1);
+                w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+                w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+                const int idx = BWD ? bwd_idx : (((i_lo + i) * BK) >> log2B) & 3;
+                a = s.amx[ws][amx_row * 4 + idx];
+            } else {
 #pragma unroll
-            for (int jj = 0; jj < WORDS; ++jj) {  // chunk j = weights 8j .. 8j+7 = bytes 4j..4j+3
-                const int j = WORDS * part + jj;
+                for (int q = 0; q < 8; ++q) w[q] = 0u;
+                a = 0.0f;
+            }
+            mbar_arrive(&s.empty_w[ws]);
+            return true;
+        };
+        uint32_t w[8], nw[8];
+        float a = 0.0f, na = 0.0f;
+        bool ok = iters > 0 && load(0, w, a);
+        for (int i = 0; i < iters && ok; ++i) {
+            const int sb = i % B_STAGES;
+            if (i + 1 < iters) ok = load(i + 1, nw, na);
+            if (i >= B_STAGES && !mbar_wait(&s.empty_b[sb], ((i / B_STAGES) - 1) & 1, abort)) break;
+            uint8_t *bt = s.b[sb];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {  // chunk j = weights 8j .. 8j+7 = bytes 4j..4j+3
                 uint32_t o[4];
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const uint32_t byte_sh = 8 * h;  // byte h of word j
-                    const float ch = __uint_as_float(shfl_idx(my_code, w[jj] >> (byte_sh + 4)));
-                    const float cl = __uint_as_float(shfl_idx(my_code, w[jj] >> byte_sh));
+                    const float ch = __uint_as_float(shfl_idx(my_code, w[j] >> (byte_sh + 4)));
+                    const float cl = __uint_as_float(shfl_idx(my_code, w[j] >> byte_sh));
                     o[h] = Dt<D>::pack2(__fmul_rn(ch, a), __fmul_rn(cl, a));
                 }
-                if (BWD || t < BN)
+                if (active)
                     *reinterpret_cast<uint4 *>(bt + swz(row_base, row_sw, j)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
             fence_proxy_async();
-            mbar_arrive(&s.full_b[st]);
+            mbar_arrive(&s.full_b[sb]);
 #pragma unroll
-            for (int q = 0; q < WORDS; ++q) w[q] = nw[q];
+            for (int q = 0; q < 8; ++q) w[q] = nw[q];
             a = na;
         }
 
@@ -423,15 +533,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
                 __syncwarp();
                 tc_fence_after();
                 // warp 2 + ew: TMEM lane quadrant warp & 3 (the one it may read),
-                // accumulator (ew >> 2) & 1, column part ew >> 3
+                // accumulator ew >> 2
                 const int ew = warp - 2;
                 const int q = warp & 3;
                 const int mt = (ew >> 2) & 1;
                 const int row = m0 + mt * 128 + q * 32 + lane;
                 const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
-                const int cbeg = (ew >> 3) * (BN / RUN_PARTS);
 #pragma unroll 1
-                for (int cc = cbeg; cc < cbeg + BN / RUN_PARTS; cc += 16) {
+                for (int cc = 0; cc < BN; cc += 16) {
                     uint32_t r[16];
                     tmem_ld16(tbase + cc, r);
                     tmem_ld_wait();
@@ -440,7 +549,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
                         float v[16];
 #pragma unroll
                         for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(r[e]);
-                        store_out<D>(out, row, n_out, col, v, 16, bias, !BWD);
+                        store_out<D, 16>(out, row, n_out, col, v, bias, !BWD);
                     }
                 }
             }
@@ -452,8 +561,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
     // barriers, whatever happened before, so none can be left waiting.
     if (C > 1) {
         __syncwarp();
+        const bool dq = warp >= 2 && warp < W_WARP;
         bool have = false;
-        if (warp >= 2) {
+        if (dq) {
             have = __all_sync(FULL, mbar_wait(&s.tmem_full, 0, abort));
             if (have) tc_fence_after();
         }
@@ -464,14 +574,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
         const int rows_per = BM / C;
 #pragma unroll 1
         for (int cb = 0; cb < BN; cb += RED_CW) {
-            if (warp >= 2 && have) {
+            if (dq && have) {
                 const int ew = warp - 2;
                 const int q = warp & 3, mt = (ew >> 2) & 1;
                 const int lrow = mt * 128 + q * 32 + lane;
                 const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
-                const int cbeg = (ew >> 3) * (RED_CW / RUN_PARTS);
 #pragma unroll
-                for (int cc = cbeg; cc < cbeg + RED_CW / RUN_PARTS; cc += 16) {
+                for (int cc = 0; cc < RED_CW; cc += 16) {
                     uint32_t r[16];
                     tmem_ld16(tbase + cb + cc, r);
                     tmem_ld_wait();
@@ -483,7 +592,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
                 }
             }
             cluster_sync_all();
-            if (warp >= 2) {
+            if (dq) {
                 const int e0 = threadIdx.x - 64;
                 for (int v = e0; v < rows_per * (RED_CW / 4); v += NUM_DQ_WARPS * 32) {
                     const int lr = z * rows_per + v / (RED_CW / 4);
@@ -497,7 +606,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__rest
                     const int row = m0 + lr, col = c0 + cb + c4;
                     if (row < M && col < n_out) {
                         const float vv[4] = {acc.x, acc.y, acc.z, acc.w};
-                        store_out<D>(out, row, n_out, col, vv, 4, bias, !BWD);
+                        store_out<D, 4>(out, row, n_out, col, vv, bias, !BWD);
                     }
                 }
             }
@@ -527,9 +636,9 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 template <typename D, bool BWD, int BN>
-cudaError_t launch_bn(const CUtensorMap &map, const uint8_t *W, const float *absmax,
-                      const void *bias, void *out, int M, int N, int K, int log2B,
-                      const CodeTable &tab, int C, cudaStream_t stream) {
+cudaError_t launch_bn(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_amx,
+                      const float *absmax, const void *bias, void *out, int M, int N, int K,
+                      int log2B, int amx_tma, const CodeTable &tab, int C, cudaStream_t stream) {
     const size_t smem = sizeof(Smem) + 1024;
     static bool attr_set = false;
     if (!attr_set) {
@@ -551,9 +660,9 @@ cudaError_t launch_bn(const CUtensorMap &map, const uint8_t *W, const float *abs
     attr[0].val.clusterDim.z = C;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<D, BWD, BN>, map, W, absmax,
+    return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<D, BWD, BN>, map_a, map_w, map_amx, absmax,
                               static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(out), M,
-                              N, K, log2B, tab);
+                              N, K, log2B, amx_tma, tab);
 }
 
 // fraction of the SM slots that the last wave of `tiles` one-SM CTAs leaves busy
@@ -562,27 +671,33 @@ double wave_eff(long tiles, int sms) {
     return (double)tiles / (double)(waves * sms);
 }
 
+CUresult encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t inner,
+                   uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swizzle) {
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+    cuuint64_t strides[1] = {(cuuint64_t)pitch_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return get_encode()(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 template <typename D, bool BWD>
 cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const void *bias,
                      void *out, int M, int N, int K, int log2B, const CodeTable &tab,
                      cudaStream_t stream) {
-    auto encode = get_encode();
-    if (!encode) return cudaErrorNotSupported;
+    if (!get_encode()) return cudaErrorNotSupported;
     const int red = BWD ? N : K;
     const int n_out = BWD ? K : N;
     // A: [M rows, red columns] row-major; TMA needs a 16-byte row pitch
     if ((red * 2) % 16 != 0) return cudaErrorInvalidValue;
-    CUtensorMap map;
-    cuuint64_t dims[2] = {(cuuint64_t)red, (cuuint64_t)M};
-    cuuint64_t strides[1] = {(cuuint64_t)red * 2};
-    cuuint32_t box[2] = {BK, 128};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = encode(&map, std::is_same<D, BF16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                        2, const_cast<void *>(A), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const CUtensorMapDataType a_type = std::is_same<D, BF16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap map_a, map_w, map_amx;
+    if (encode_2d(&map_a, a_type, A, red, M, (uint64_t)red * 2, BK, 128, CU_TENSOR_MAP_SWIZZLE_128B) !=
+        CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
 
     const int sms = device_sm_count();
     const long mt = (M + BM - 1) / BM;
@@ -591,6 +706,25 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
     int bn = 256;
     if (!BWD && wave_eff(mt * ((n_out + 223) / 224), sms) > wave_eff(mt * ((n_out + 255) / 256), sms) + 0.02)
         bn = 224;
+    // packed weights [N rows, K/2 bytes]: per stage BN rows x 32 bytes (forward)
+    // or 64 rows x 128 bytes (backward)
+    const uint64_t row_bytes = (uint64_t)K / 2;  // a multiple of 16: K % 32 == 0
+    const CUresult rw =
+        BWD ? encode_2d(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, row_bytes, N, row_bytes, BN_MAX / 2, BK,
+                        CU_TENSOR_MAP_SWIZZLE_128B)
+            : encode_2d(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, row_bytes, N, row_bytes, BK / 2, bn,
+                        CU_TENSOR_MAP_SWIZZLE_32B);
+    if (rw != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    // absmax [N rows, K / blocksize]: 16-byte boxes when its row pitch allows,
+    // otherwise gathered by the producer warp
+    const int nblk = K >> log2B;
+    int amx_tma = (nblk % 4 == 0) ? 1 : 0;
+    memset(&map_amx, 0, sizeof(map_amx));
+    if (amx_tma &&
+        encode_2d(&map_amx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, absmax, nblk, N, (uint64_t)nblk * 4, 4,
+                  BWD ? BK : bn, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        amx_tma = 0;
+
     const long tiles = mt * ((n_out + bn - 1) / bn);
     // split the reduction over a cluster when the tiles alone leave SMs idle
     // and every CTA keeps at least 16 stages
@@ -599,9 +733,11 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
     while (C < 8 && tiles * (2 * C) <= sms && iters / (2 * C) >= 16) C *= 2;
     if constexpr (!BWD) {
         if (bn == 224)
-            return launch_bn<D, BWD, 224>(map, W, absmax, bias, out, M, N, K, log2B, tab, C, stream);
+            return launch_bn<D, BWD, 224>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B,
+                                          amx_tma, tab, C, stream);
     }
-    return launch_bn<D, BWD, 256>(map, W, absmax, bias, out, M, N, K, log2B, tab, C, stream);
+    return launch_bn<D, BWD, 256>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma,
+                                  tab, C, stream);
 }
 
 }  // namespace

@@ -105,7 +105,7 @@ template <typename D>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-            uint16_t *__restrict__ y, int N, int K, int log2B, CodeTable tab) {
+            uint16_t *__restrict__ y, int N, int K, int log2B, const __grid_constant__ CodeTable tab) {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
     uint8_t *ring = smem + kLut;                                                  // warps x STAGES

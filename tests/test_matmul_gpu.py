@@ -119,10 +119,12 @@ def _ref_backward(Wt, dYs, dt, M, entries=None):
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 @pytest.mark.parametrize("M,N,K,B", [(17, 256, 256, 64), (100, 320, 512, 64), (256, 512, 1024, 128),
                                      (300, 96, 256, 256), (257, 264, 704, 64), (300, 256, 4096, 64),
-                                     (300, 33152, 256, 64)])
+                                     (300, 33152, 256, 64), (300, 33152, 192, 64)])
 def test_gemm_large_m(q, dt, M, N, K, B):
-    """Includes a reduction split over a cluster (K=4096, two tiles) and a width
-    (N = 148 * 224) where 224-column tiles fill the SMs."""
+    """Includes a reduction split over a cluster (K=4096, two tiles), a width
+    (N = 148 * 224) where 224-column tiles fill the SMs, and absmax rows whose
+    pitch (K / B scales) is not a multiple of four (K = 704, 192 at B = 64;
+    K = 256 at B = 256)."""
     Wt = Weight(N, K, B, q, seed=M)
     Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
     bs = synthetic.storage_numpy(synthetic.bias(N, seed=2, dtype=dt)) if M % 2 == 0 else None
@@ -137,9 +139,13 @@ def test_gemm_large_m(q, dt, M, N, K, B):
 @pytest.mark.parametrize("dt", ["bf16", "f16"])
 @pytest.mark.parametrize("M,N,K,B", [(1, 256, 256, 64), (17, 256, 512, 64), (256, 200, 256, 64),
                                      (300, 320, 768, 256), (64, 1024, 1280, 128),
-                                     (64, 8192, 256, 64), (300, 4096, 512, 128)])
+                                     (64, 8192, 256, 64), (300, 4096, 512, 128),
+                                     (130, 264, 2048, 128), (96, 520, 3072, 512)])
 def test_gemm_backward(q, dt, M, N, K, B):
-    """Includes reductions long enough to be split over a thread-block cluster."""
+    """Includes reductions long enough to be split over a thread-block cluster,
+    ragged reductions (N = 200, 264, 520), blocks of 128 scales shared by two
+    64-column groups of a tile, and absmax pitches that are not a multiple of
+    four scales (K / B = 3, 10, 6)."""
     Wt = Weight(N, K, B, q, seed=N)
     dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3, dtype=dt)).reshape(-1)
     dX = bnb4.gemm_4bit_backward(to_dev(dYs, dt).view(M, N), Wt.dp, Wt.da, K, B, q)

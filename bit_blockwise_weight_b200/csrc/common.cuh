@@ -67,6 +67,50 @@ struct CodeTable {
 // Host-side construction (also used to build the decision tables).
 CodeTable host_code_table(bnb4_quant_type qt);
 
+// ------------------------------------------- decode by byte permutation
+//
+// Dequantizing a run of one block without shuffles or table loads: the 16
+// values RN_dtype(fp32(code_i * absmax)) are computed once per block and held
+// as two byte planes (lo[q]: low bytes of entries 4q..4q+3; hi[q]: high
+// bytes), from which prmt selects four entries at a time.  The values are the
+// ones a per-element __fmul_rn followed by the dtype conversion produces.
+
+struct ScaledPlanes {
+    uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+template <typename D>
+__device__ __forceinline__ ScaledPlanes scaled_planes(const CodeTable &tab, float a) {
+    ScaledPlanes s;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t p0 = Dt<D>::pack2(__fmul_rn(tab.v[4 * q], a), __fmul_rn(tab.v[4 * q + 1], a));
+        const uint32_t p1 = Dt<D>::pack2(__fmul_rn(tab.v[4 * q + 2], a), __fmul_rn(tab.v[4 * q + 3], a));
+        s.lo[q] = prmt(p0, p1, 0x6420u);
+        s.hi[q] = prmt(p0, p1, 0x7531u);
+    }
+    return s;
+}
+
+// The four codes in the low 16 bits of x (two packed bytes, the first element
+// of each byte in its high nibble) -> o0 = (e0, e1), o1 = (e2, e3), the first
+// element of each pair in the low half.
+__device__ __forceinline__ void decode4(const ScaledPlanes &s, uint32_t x, uint32_t &o0, uint32_t &o1) {
+    const uint32_t sel = x & 0x7777u;                     // byte k <- entry (nibble k) & 7
+    const uint32_t f = ((x >> 1) & 0x4444u) | 0x3210u;    // entries 8..15 where bit 3 is set
+    const uint32_t rl = prmt(prmt(s.lo[0], s.lo[1], sel), prmt(s.lo[2], s.lo[3], sel), f);
+    const uint32_t rh = prmt(prmt(s.hi[0], s.hi[1], sel), prmt(s.hi[2], s.hi[3], sel), f);
+    // rl, rh list the nibbles in register order: e1, e0, e3, e2
+    o0 = prmt(rl, rh, 0x4051u);
+    o1 = prmt(rl, rh, 0x6273u);
+}
+
 // ------------------------------------------------------ decision tables
 //
 // Nearest-code search without a 16-way compare.  v in [-1, 1] falls into one
@@ -80,7 +124,21 @@ CodeTable host_code_table(bnb4_quant_type qt);
 struct QuantTables {
     float thr[32];
     uint32_t lohi[32];
+    // One-shuffle screen.  key[k]: the threshold of cell k with its low four
+    // mantissa bits replaced by the rank (position in ascending value order)
+    // just above it, or -2^100 with the low bits holding the cell's only
+    // rank.  The replacement moves a threshold by less than 2^-20, so an
+    // element whose approximate quotient lies further than kNear from the key
+    // decides exactly as its exact quotient would (rank = key & 15, less one
+    // below the key); the others are redone exactly, with rank_lohi[k] = rank
+    // below | rank above << 4.  fast: 0 = exact search only, 1 = ranks are
+    // code indices, 2 = ranks map to code indices by the E2M1 fold
+    // (r >= 7 ? r - 7 : 15 - r).
+    uint32_t key[32];
+    uint32_t rank_lohi[32];
+    int fast;
 };
+constexpr float kNear = 0x1p-19f;
 
 QuantTables host_quant_tables(bnb4_quant_type qt);
 

@@ -21,7 +21,8 @@
 //     a 4-slot ring.  When the absmax row pitch is not a multiple of 16 bytes
 //     the warp gathers the absmax values with ordinary loads instead;
 //   * warps 2-9: each thread reads one 64-element weight run (32 packed bytes
-//     + its block absmax) from the ring, decodes it and writes one 128-byte row
+//     + its block absmax) from the ring, decodes it by byte permutation from
+//     the block's 16 scaled values (no shuffles) and writes one 128-byte row
 //     of the B tile in the canonical 128-byte-swizzled layout: K-major rows for
 //     the forward, MN-major rows for the backward (so neither needs a
 //     transpose), fences the writes to the async proxy and arrives on the stage
@@ -42,6 +43,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 #include <type_traits>
 
@@ -190,14 +192,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t shfl_idx(uint32_t v, uint32_t lane_bits) {
-    uint32_t r;
-    asm volatile("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;"
-                 : "=r"(r)
-                 : "r"(v), "r"(lane_bits));
-    return r;
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm100 version 1.
@@ -452,7 +446,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
         // ---------------------------------------- weight dequant warps
         // 256 runs of 64 weights per stage, one per thread
         const int t = threadIdx.x - 64;
-        const uint32_t my_code = __float_as_uint(tab.v[lane & 15]);
         // forward: row t of the tile (output column c0 + t) over the stage's 64
         // reduction indices; backward: reduction row (t & 63) of the stage over
         // output columns c0 + 64 (t >> 6) ... + 63
@@ -506,16 +499,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
             if (i + 1 < iters) ok = load(i + 1, nw, na);
             if (i >= B_STAGES && !mbar_wait(&s.empty_b[sb], ((i / B_STAGES) - 1) & 1, abort)) break;
             uint8_t *bt = s.b[sb];
+            const ScaledPlanes sp = scaled_planes<D>(tab, a);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {  // chunk j = weights 8j .. 8j+7 = bytes 4j..4j+3
                 uint32_t o[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const uint32_t byte_sh = 8 * h;  // byte h of word j
-                    const float ch = __uint_as_float(shfl_idx(my_code, w[j] >> (byte_sh + 4)));
-                    const float cl = __uint_as_float(shfl_idx(my_code, w[j] >> byte_sh));
-                    o[h] = Dt<D>::pack2(__fmul_rn(ch, a), __fmul_rn(cl, a));
-                }
+                decode4(sp, w[j], o[0], o[1]);
+                decode4(sp, w[j] >> 16, o[2], o[3]);
                 if (active)
                     *reinterpret_cast<uint4 *>(bt + swz(row_base, row_sw, j)) = make_uint4(o[0], o[1], o[2], o[3]);
             }
@@ -581,6 +570,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                 const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
 #pragma unroll
                 for (int cc = 0; cc < RED_CW; cc += 16) {
+                    if (cb + cc >= BN) break;  // a 224-wide tile ends inside the last chunk
                     uint32_t r[16];
                     tmem_ld16(tbase + cb + cc, r);
                     tmem_ld_wait();
@@ -597,12 +587,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                 for (int v = e0; v < rows_per * (RED_CW / 4); v += NUM_DQ_WARPS * 32) {
                     const int lr = z * rows_per + v / (RED_CW / 4);
                     const int c4 = (v % (RED_CW / 4)) * 4;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (cb + c4 >= BN) continue;
                     const uint32_t la = stg_addr + (uint32_t)(lr * RED_PITCH + c4) * 4;
-                    for (int q2 = 0; q2 < C; ++q2) {
-                        const float4 p = ld_dsmem_f4(la, (uint32_t)q2);
-                        acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
-                    }
+                    // all C partials in flight before the first add (C <= 8)
+                    float4 p[8];
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2)
+                        if (q2 < C) p[q2] = ld_dsmem_f4(la, (uint32_t)q2);
+                    float4 acc = p[0];
+#pragma unroll
+                    for (int q2 = 1; q2 < 8; ++q2)
+                        if (q2 < C) {
+                            acc.x += p[q2].x; acc.y += p[q2].y; acc.z += p[q2].z; acc.w += p[q2].w;
+                        }
                     const int row = m0 + lr, col = c0 + cb + c4;
                     if (row < M && col < n_out) {
                         const float vv[4] = {acc.x, acc.y, acc.z, acc.w};
@@ -635,40 +632,100 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
 template <typename D, bool BWD, int BN>
-cudaError_t launch_bn(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_amx,
-                      const float *absmax, const void *bias, void *out, int M, int N, int K,
-                      int log2B, int amx_tma, const CodeTable &tab, int C, cudaStream_t stream) {
-    const size_t smem = sizeof(Smem) + 1024;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<D, BWD, BN>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    const int n_out = BWD ? K : N;
+cudaError_t set_smem_attr() {
+    static std::atomic<bool> done{false};
+    if (done.load(std::memory_order_relaxed)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<D, BWD, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e == cudaSuccess) done.store(true, std::memory_order_relaxed);
+    return e;
+}
+
+cudaLaunchConfig_t make_cfg(dim3 grid, int C, cudaStream_t stream, cudaLaunchAttribute *attr) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((n_out + BN - 1) / BN, (M + BM - 1) / BM, C);
+    cfg.gridDim = grid;
     cfg.blockDim = dim3(THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = C;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    return cfg;
+}
+
+// CTAs of clusters of C (1, 2, 4, 8) that can be resident at once on the
+// current device: clusters must fit inside one GPC, so this can be below the
+// SM count.  Queried once per device and cluster size.
+template <typename D, bool BWD, int BN>
+int cluster_capacity(int C) {
+    static std::atomic<int> cache[64][4];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    const int ci = C == 1 ? 0 : C == 2 ? 1 : C == 4 ? 2 : 3;
+    int v = cache[dev][ci].load(std::memory_order_relaxed);
+    if (v == 0) {
+        int n = 0;
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = make_cfg(dim3(1, 1, C), C, 0, attr);
+        if (set_smem_attr<D, BWD, BN>() != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<D, BWD, BN>, &cfg) != cudaSuccess || n <= 0) {
+            (void)cudaGetLastError();
+            n = device_sm_count() / C;
+        }
+        v = n * C;
+        cache[dev][ci].store(v, std::memory_order_relaxed);
+    }
+    return v;
+}
+
+template <typename D, bool BWD, int BN>
+cudaError_t launch_bn(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_amx,
+                      const float *absmax, const void *bias, void *out, int M, int N, int K,
+                      int log2B, int amx_tma, const CodeTable &tab, int C, cudaStream_t stream) {
+    cudaError_t e = set_smem_attr<D, BWD, BN>();
+    if (e != cudaSuccess) return e;
+    const int n_out = BWD ? K : N;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = make_cfg(dim3((n_out + BN - 1) / BN, (M + BM - 1) / BM, C), C, stream, attr);
     return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<D, BWD, BN>, map_a, map_w, map_amx, absmax,
                               static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(out), M,
                               N, K, log2B, amx_tma, tab);
 }
 
-// fraction of the SM slots that the last wave of `tiles` one-SM CTAs leaves busy
-double wave_eff(long tiles, int sms) {
-    const long waves = (tiles + sms - 1) / sms;
-    return (double)tiles / (double)(waves * sms);
+// Tile width and reduction split: the pair minimising
+//   waves x (stages per CTA + fixed cost) x width / 256,
+// the fixed cost (prologue, epilogue; the cluster reduction when split) in
+// stage units.  A split keeps at least 8 stages per CTA.
+struct Plan {
+    int bn, C;
+};
+
+template <typename D, bool BWD>
+Plan make_plan(long mt, int n_out, int iters) {
+    Plan best{256, 1};
+    double best_t = 1e300;
+    for (int bn : {256, 224}) {
+        if (BWD && bn == 224) continue;  // the MN-major tile is built from 64-column atoms
+        const long tiles = mt * ((n_out + bn - 1) / bn);
+        for (int C = 1; C <= 8; C *= 2) {
+            if (C > 1 && iters / C < 8) break;
+            const int cap = bn == 256 ? cluster_capacity<D, BWD, 256>(C)
+                                      : cluster_capacity<D, BWD, BWD ? 256 : 224>(C);
+            const long waves = (tiles * C + cap - 1) / cap;
+            const double t = (double)waves * ((iters + C - 1) / C + (C == 1 ? 4 : 8)) * bn / 256.0;
+            if (t < best_t - 1e-9) {
+                best_t = t;
+                best = Plan{bn, C};
+            }
+        }
+    }
+    return best;
 }
 
 CUresult encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t inner,
@@ -699,13 +756,10 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
         CUDA_SUCCESS)
         return cudaErrorInvalidValue;
 
-    const int sms = device_sm_count();
     const long mt = (M + BM - 1) / BM;
-    // tile width: 224 when it fills the SMs better (forward only; the backward's
-    // MN-major weight tile is built from 64-column atoms)
-    int bn = 256;
-    if (!BWD && wave_eff(mt * ((n_out + 223) / 224), sms) > wave_eff(mt * ((n_out + 255) / 256), sms) + 0.02)
-        bn = 224;
+    const int iters = (red + BK - 1) / BK;
+    const Plan plan = make_plan<D, BWD>(mt, n_out, iters);
+    const int bn = plan.bn, C = plan.C;
     // packed weights [N rows, K/2 bytes]: per stage BN rows x 32 bytes (forward)
     // or 64 rows x 128 bytes (backward)
     const uint64_t row_bytes = (uint64_t)K / 2;  // a multiple of 16: K % 32 == 0
@@ -725,12 +779,6 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
                   BWD ? BK : bn, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
         amx_tma = 0;
 
-    const long tiles = mt * ((n_out + bn - 1) / bn);
-    // split the reduction over a cluster when the tiles alone leave SMs idle
-    // and every CTA keeps at least 16 stages
-    const int iters = (red + BK - 1) / BK;
-    int C = 1;
-    while (C < 8 && tiles * (2 * C) <= sms && iters / (2 * C) >= 16) C *= 2;
     if constexpr (!BWD) {
         if (bn == 224)
             return launch_bn<D, BWD, 224>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B,

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -80,7 +81,35 @@ QuantTables host_quant_tables(bnb4_quant_type qt) {
         const int hi = inside >= 0 ? idx[base + 1] : lo;
         q.thr[k] = inside >= 0 ? thr[inside] : 2.0f;  // 2 > every |v| <= 1
         q.lohi[k] = (uint32_t)lo | ((uint32_t)hi << 4);
+        uint32_t key;
+        if (inside >= 0) {
+            std::memcpy(&key, &thr[inside], 4);
+            key = (key & ~15u) | (uint32_t)(base + 1);
+        } else {
+            const float below_all = -0x1p100f;
+            std::memcpy(&key, &below_all, 4);
+            key |= (uint32_t)base;
+        }
+        q.key[k] = key;
+        q.rank_lohi[k] = (uint32_t)base | ((uint32_t)(inside >= 0 ? base + 1 : base) << 4);
     }
+    // The screen is exact when (a) every threshold lies in (-1, 1), so the
+    // key moves it by less than 16 ulp <= 2^-20, and (b) no threshold lies
+    // within 2^-16 of a cell boundary (j - 12.5) / 13, so a cell index taken
+    // from an approximate quotient (relative error ~2^-22) can only differ
+    // from the exact one where the nearest code does not change.
+    bool ok = true;
+    for (int r = 0; r + 1 < nd; ++r) {
+        if (!(std::fabs(thr[r]) < 1.0f)) ok = false;
+        for (int j = 0; j <= 26; ++j)
+            if (std::fabs((double)thr[r] - (j - 12.5) / 13.0) <= 0x1p-16) ok = false;
+    }
+    bool ident = true, fold = true;
+    for (int r = 0; r < nd; ++r) {
+        if (idx[r] != r) ident = false;
+        if (idx[r] != (r >= 7 ? r - 7 : 15 - r)) fold = false;
+    }
+    q.fast = !ok ? 0 : ident ? 1 : fold ? 2 : 0;
     return q;
 }
 

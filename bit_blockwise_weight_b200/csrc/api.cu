@@ -121,9 +121,8 @@ bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, cons
                       bnb4_dtype dt, cudaStream_t stream) {
     bnb4_status s = check_matmul(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt);
     if (s != BNB4_OK) return s;
-    // small M streams the weight once per call; the per-CTA row range of that
-    // kernel is capped at 1024 rows, beyond which the tensor-core kernel takes over
-    if (M <= kSmallMMax && N <= (int64_t)device_sm_count() * 1024)
+    // small M: one pass over the weight stream, decoded into tensor memory
+    if (M <= kSmallMMax)
         return from_cuda(launch_gemm_small(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, stream));
     return from_cuda(launch_gemm_tc(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, false, stream));
 }

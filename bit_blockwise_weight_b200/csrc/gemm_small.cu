@@ -1,47 +1,86 @@
-// gemm_small.cu -- gemm_4bit for small M (1 <= M <= 16): Y = X @ dequant(W)^T (+ bias).
+// gemm_small.cu -- gemm_4bit for 1 <= M <= 16, gemv included:
+// Y[M, N] = X[M, K] . dequant(W)[N, K]^T (+ bias).
 //
-// "Feat/mps gemm 4bit bf16", What runs natively now (gemm_4bit, general M)
-// and Performance (small M is dominated by the weight stream).  At M <= 16
-// the product is a real matrix-matrix product, but it still moves 0.5625 B
-// of weight per 2*M flops, far below the tensor-core ridge: the weight stream
-// sets the time.  CUDA-core FMAs cannot keep up with 16 products per decoded
-// weight, so the decoded weights go straight from registers into
-// mma.sync.m16n8k16 fragments (W is the 16-row A operand, X^T the 8-column B
-// operand), with fp32 accumulation.
+// "Feat/mps gemm 4bit bf16", What runs natively now (gemv_4bit for M == 1 and
+// gemm_4bit for general M) and Performance (small M is dominated by the
+// weight stream).  At M <= 16 the product moves 0.5625 B of weight per 2 M
+// flops: the weight stream sets the time, and decoding the 4-bit codes at HBM
+// rate is the work.  Weight tiles are small and many, so the multiply-adds go
+// to mma.sync.m16n8k16 fed straight from registers (W is the 16-row A operand,
+// X^T the 8-column B operand, fp32 accumulation):
 //
-// Decode: a 256-entry table maps one packed byte to the two codes it holds
-// as a bf16x2 / f16x2 register (first element in the low half).  The table is
-// replicated once per shared-memory bank (32 KB) so that every lane reads its
-// own bank: lookups never conflict.
+//   * warp 0 streams, per four 64-element runs of K, the CTA's packed-weight
+//     tile (rows x 128 bytes, 128-byte swizzle), its absmax tile and four
+//     16-token X tiles (64 elements each, 128-byte swizzle; tokens past M
+//     arrive as zeros) into a 4-slot ring with TMA;
+//   * warps 1-16 each own one 16-row tile of the CTA's rows.  Per run a lane
+//     reads its 8 packed bytes of two rows and its X fragments with
+//     conflict-free shared loads, turns each byte into a pair of 16-bit codes
+//     through a byte table replicated once per shared-memory bank, and issues
+//     the MMAs; the run's sums are scaled by the block absmax in fp32.
 //
-// K order inside a 64-element quantization block: lane (g, t) owns weights
-// [16t, 16t+16) of rows g and g+8 (8 contiguous bytes each).  For mma step s
-// (0..3) it feeds bytes 2s and 2s+1 of its 8, so k-slot 2t+e holds
-// k = 16t + 4s + e and k-slot 2t+8+e holds k = 16t + 4s + 2 + e; the B
-// fragment takes the same k values of X.  The reduction over k is a plain sum,
-// so the order is free, and every step stays inside one block: the four steps
-// of a block accumulate into a block sum that is scaled by the block's absmax
-// in fp32 once.
+// K order inside a 64-element run: lane (g, t) owns weights [16t, 16t+16) of
+// rows g and g+8 (8 contiguous bytes each).  For mma step s (0..3) it feeds
+// bytes 2s and 2s+1 of its 8, so k-slot 2t+e holds k = 16t + 4s + e and k-slot
+// 2t+8+e holds k = 16t + 4s + 2 + e; the B fragment takes the same k values of
+// X.  The reduction over k is a plain sum, so the order is free, and every
+// step stays inside one run, hence one block.  So the weight a token meets is
+// RN_dtype(code) * absmax, accumulated in fp32; the codes, as 16-bit values,
+// lose at most 2^-9 (bf16) or 2^-12 (f16) relative.
 //
-// Work split (persistent, one CTA per SM): CTA c owns rows
-// [N c / G, N (c+1) / G) -- balanced to one row -- and all of K.  Its rows form
-// T tiles of 16 (the last one partial), grouped by up to 4 per warp so that
-// each X fragment feeds 4 tiles; the 8 warps split the groups and then K.
-// Weights, absmax and X fragments of the next block are loaded into registers
-// while the current block is multiplied.  Partial sums of the warps that
-// share a group meet in shared memory.  No global scratch.
+// Work split: CTA (g, z) owns rows [N g / G, N (g+1) / G) (balanced to one
+// row, at most 256) and the z-th of S shares of the K stages; the S CTAs of a
+// cluster add their partial sums through distributed shared memory.  No
+// global scratch.  Every mbarrier wait is bounded.
+#include <atomic>
+#include <cstring>
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace bnb4 {
 
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int MT = 4;                 // m16 tiles per warp
-constexpr int kMaxTiles = 64;         // rows per CTA <= 1024
-constexpr int kMaxM = 16;
+constexpr int kRowsMax = 256;                     // weight rows per CTA
+constexpr int RUN = 64;                           // weights per row per run (one block or less)
+constexpr int RPS = 4;                            // runs per stage (128-byte weight rows)
+constexpr int STAGES = 4;
+constexpr int NTOK = 16;                          // tokens, zero-padded
+constexpr int W_SLOT = kRowsMax * RPS * RUN / 2;  // 32 KB
+constexpr int X_RUN = NTOK * RUN * 2;             // 2 KB per run
+constexpr int X_SLOT = RPS * X_RUN;               // 8 KB
+constexpr int AMX_SLOT = kRowsMax * 4;            // one 16-byte box per row
+constexpr int NCW = 16;                           // compute warps (one 16-row tile each)
+constexpr int MT = kRowsMax / 16 / NCW;           // 16-row tiles per compute warp
+constexpr int THREADS = (1 + NCW) * 32;           // 544
+
+struct Smem {
+    uint8_t w[STAGES][W_SLOT];   // 1024-byte aligned (128-byte swizzle atoms)
+    uint8_t x[STAGES][X_SLOT];   // 1024-byte aligned
+    float amx[STAGES][AMX_SLOT];
+    uint64_t full[STAGES], empty[STAGES];
+    int abort;
+};
+static_assert(kRowsMax * NTOK * 4 <= STAGES * W_SLOT, "output staging fits in the weight ring");
+static_assert(sizeof(Smem) + 1024 + 256 * 32 * 4 <= 227 * 1024, "shared memory plan");
+
+// byte -> (code hi nibble, code lo nibble) as a 16-bit pair, one copy per
+// bank: entry e of lane l at word 32 e + l
+__shared__ uint32_t s_lut[256 * 32];
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
 
 template <typename D> struct Mma;
 template <> struct Mma<BF16> {
@@ -61,218 +100,319 @@ template <> struct Mma<F16> {
     }
 };
 
-__device__ __forceinline__ uint2 ld_stream8(const uint8_t *p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
-
-// byte j (0..3) of a word -> offset of its entry in this lane's bank
-// (entry e of lane l sits at word 32 e + l)
-__device__ __forceinline__ uint32_t lut_off(uint32_t w, int j, uint32_t lane4) {
+// offset of byte j (0..3) of w's table entry in this lane's bank
+__device__ __forceinline__ uint32_t lut_off(uint32_t w, int j) {
     const uint32_t sh = j == 0 ? (w << 7) : (w >> (8 * j - 7));
-    return (sh & 0x7f80u) | lane4;
+    return sh & 0x7f80u;
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
-
-struct Frag {
-    uint2 w[MT][2];     // rows g and g+8 of each tile: 8 bytes (16 weights)
-    float a[MT][2];     // their block absmax
-};
-
+// NT = 1 for M <= 8 (tokens 0..7), 2 for M <= 16
 template <typename D, int NT>
-__global__ void __launch_bounds__(kThreads, 1)
-gemm_small_kernel(const uint16_t *__restrict__ X, const uint8_t *__restrict__ W,
-                  const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-                  uint16_t *__restrict__ Y, int M, int N, int K, int log2B, const __grid_constant__ CodeTable tab) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *lut = reinterpret_cast<uint32_t *>(smem);                 // 256 x 32 words
-    float *sum = reinterpret_cast<float *>(smem + 256 * 32 * 4);        // [kMaxTiles*16][16]
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_amx,
+                  const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ absmax,
+                  const uint16_t *__restrict__ bias, uint16_t *__restrict__ Y, int M, int N, int K,
+                  int log2B, int amx_tma, int rbox, const __grid_constant__ CodeTable tab) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~(uintptr_t)1023);
+    volatile int *abort = &s.abort;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, t = lane & 3;
-
-    // CTA rows
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x;
-    const int r0 = (int)(((int64_t)N * blockIdx.x) / G);
-    const int r1 = (int)(((int64_t)N * (blockIdx.x + 1)) / G);
-    const int T = (r1 - r0 + 15) >> 4;  // tiles
-    const int nb = K >> 6;              // 64-element blocks along K
-    const int64_t row_bytes = K >> 1;
+    const int r0 = (int)(((int64_t)N * blockIdx.x) / G), r1 = (int)(((int64_t)N * (blockIdx.x + 1)) / G);
+    const int R = r1 - r0;
+    const int S = gridDim.z, z = blockIdx.z;
+    const int nb = K / RUN;
+    // K split in whole stages, so that a stage's absmax box starts on a
+    // 4-scale boundary
+    const int nq = (nb + RPS - 1) / RPS;
+    const int b_lo = RPS * (int)(((int64_t)nq * z) / S);
+    const int b_hi = min(nb, RPS * (int)(((int64_t)nq * (z + 1)) / S));
+    const int iters = b_hi > b_lo ? b_hi - b_lo : 0;  // runs
+    const int stages = (iters + RPS - 1) / RPS;
     const int nblk = K >> log2B;
 
-    // byte -> code pair table, one copy per bank (a thread fills 4 copies at once)
-    for (int e = tid >> 3; e < 256; e += kThreads / 8) {
-        const uint32_t v = Dt<D>::pack2(tab.v[e >> 4], tab.v[e & 15]);
-        reinterpret_cast<uint4 *>(lut + e * 32)[tid & 7] = make_uint4(v, v, v, v);
+    for (int e = threadIdx.x; e < 256 * 8; e += THREADS) {  // one entry's copies for 4 lanes
+        const uint32_t v = Dt<D>::pack2(tab.v[(e >> 3) >> 4], tab.v[(e >> 3) & 15]);
+        reinterpret_cast<uint4 *>(s_lut)[e] = make_uint4(v, v, v, v);
     }
-    for (int e = tid; e < T * 16 * kMaxM; e += kThreads) sum[e] = 0.f;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], NCW);  // one arrival per compute warp
+        }
+        s.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     __syncthreads();
-    if (T == 0) return;
 
-    const uint32_t lut_base = (uint32_t)__cvta_generic_to_shared(lut);
-    const uint32_t lane4 = 4u * lane;
+    float acc[MT][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.0f;
+    const int g = lane >> 2, t = lane & 3, wc = warp - 1;
 
-    // warp -> (tile group, K part)
-    const int groups = (T + MT - 1) / MT;
-    for (int gbase = 0; gbase < groups; gbase += kWarps) {
-        const int gcount = min(kWarps, groups - gbase);
-        const int kparts = kWarps / gcount;
-        const int gi = gbase + warp / kparts;
-        const int kp = warp % kparts;
-        const bool active = warp < gcount * kparts;
-        const int b_lo = active ? (int)(((int64_t)nb * kp) / kparts) : 0;
-        const int b_hi = active ? (int)(((int64_t)nb * (kp + 1)) / kparts) : 0;
-
-        int rows[MT][2];
-        bool rv[MT][2];
+    if (warp == 0) {
+        // ------------------------------------ TMA producer: weights, X, absmax
+        const uint32_t tx = (uint32_t)rbox * (RPS * RUN / 2) + X_SLOT + (amx_tma ? (uint32_t)rbox * 16u : 0u);
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
+        }
+        int issued = 0;
+        for (int q = 0; q < stages; ++q) {
+            const int st = q % STAGES;
+            bool ok = true;
+            if (q >= STAGES) ok = mbar_wait(&s.empty[st], ((q / STAGES) - 1) & 1, abort);
+            if (!__all_sync(FULL, ok)) break;
+            const int b = b_lo + q * RPS;                  // first run of the stage
+            const int x0 = ((b * RUN) >> log2B) & ~3;      // first scale of the absmax box
+            if (!amx_tma)  // absmax rows not 16-byte pitched: gather the stage's scales
+                for (int p = lane; p < R; p += 32)
+                    for (int j = 0; j < RPS && b + j < b_hi; ++j) {
+                        const int blk = ((b + j) * RUN) >> log2B;
+                        s.amx[st][p * 4 + (blk - x0)] = __ldg(absmax + (int64_t)(r0 + p) * nblk + blk);
+                    }
+            __syncwarp();  // the gathered scales are written before lane 0 arrives
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&s.full[st], tx);
+                tma_load_2d(&tmap_w, &s.full[st], s.w[st], b * (RUN / 2), r0);
+#pragma unroll
+                for (int j = 0; j < RPS; ++j)  // runs past K arrive as zeros
+                    tma_load_2d(&tmap_x, &s.full[st], s.x[st] + j * X_RUN, (b + j) * RUN, 0);
+                if (amx_tma) tma_load_2d(&tmap_amx, &s.full[st], s.amx[st], x0, r0);
+            }
+            issued = q + 1;
+        }
+        if (lane == 0)
+            for (int q = (issued > STAGES ? issued - STAGES : 0); q < issued; ++q)
+                mbar_drain(&s.full[q % STAGES], (q / STAGES) & 1);
+    } else {
+        // ------------------------------------------------ compute warps
+        const uint32_t lut = smem_u32(s_lut) + 4u * lane;
+        const uint32_t w_base = smem_u32(s.w[0]), x_base = smem_u32(s.x[0]), amx_base = smem_u32(s.amx[0]);
+        // tiles of this warp present in the CTA's rows
+        int ntl = 0;
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
+            if (16 * (wc + NCW * mt) < R) ntl = mt + 1;
+        for (int q = 0; q < stages; ++q) {
+            const int st = q % STAGES;
+            if (!__all_sync(FULL, mbar_wait(&s.full[st], (q / STAGES) & 1, abort))) break;
+            const int b = b_lo + q * RPS;
+            const int x0 = ((b * RUN) >> log2B) & ~3;
+            const uint32_t ws = w_base + st * W_SLOT, xs = x_base + st * X_SLOT, as = amx_base + st * (AMX_SLOT * 4);
+#pragma unroll 1
+            for (int j = 0; j < RPS; ++j) {
+                if (b + j >= b_hi) break;
+                // X fragments of run j: token nt*8 + g, k = 16t + 4s .. +3 (8 bytes)
+                uint2 xf[4][NT];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                rows[mt][h] = r0 + 16 * (gi * MT + mt) + 8 * h + g;
-                rv[mt][h] = active && (gi * MT + mt) < T && rows[mt][h] < r1;
-            }
-        auto fetch = [&](int b, Frag &f) {
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int m = nt * 8 + g;
+                    const uint32_t row = xs + j * X_RUN + (m >> 3) * 1024 + (m & 7) * 128;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    if (rv[mt][h]) {
-                        const int64_t rb = (int64_t)rows[mt][h];
-                        f.w[mt][h] = ld_stream8(W + rb * row_bytes + 32 * b + 8 * t);
-                        f.a[mt][h] = __ldg(absmax + rb * nblk + ((64 * b) >> log2B));
-                    } else {
-                        f.w[mt][h] = make_uint2(0, 0);
-                        f.a[mt][h] = 0.f;
-                    }
+                    for (int s4 = 0; s4 < 4; ++s4)
+                        xf[s4][nt] = lds64(row + ((((uint32_t)(2 * t + (s4 >> 1))) ^ (uint32_t)(m & 7)) << 4) +
+                                           8 * (s4 & 1));
                 }
-        };
-        // X fragment of block b: lane (g, t) needs X[nt*8 + g][64b + 16t + 4s .. +4] for s = 0..3
-        auto fetch_x = [&](int b, uint2 (&xf)[4][NT]) {
+                const uint32_t aoff = 4u * (uint32_t)((((b + j) * RUN) >> log2B) - x0);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int m = nt * 8 + g;
+                for (int mt = 0; mt < MT; ++mt) {
+                    if (mt >= ntl) break;
+                    const int rr0 = 16 * (wc + NCW * mt) + g, rr1 = rr0 + 8;
+                    const uint32_t chunk = (uint32_t)(2 * j + (t >> 1));
+                    const uint2 w0 = lds64(ws + rr0 * 128 + ((chunk ^ (uint32_t)(rr0 & 7)) << 4) + 8 * (t & 1));
+                    const uint2 w1 = lds64(ws + rr1 * 128 + ((chunk ^ (uint32_t)(rr1 & 7)) << 4) + 8 * (t & 1));
+                    const float a0 = __uint_as_float(lds32(as + rr0 * 16 + aoff));
+                    const float a1 = __uint_as_float(lds32(as + rr1 * 16 + aoff));
+                    float blk[NT][4];
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    xf[s][nt] = (m < M) ? __ldg(reinterpret_cast<const uint2 *>(
-                                              X + (int64_t)m * K + 64 * b + 16 * t + 4 * s))
-                                        : make_uint2(0, 0);
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) blk[nt][i] = 0.0f;
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4) {
+                        const int wi = s4 >> 1, j0 = 2 * (s4 & 1), j1 = j0 + 1;
+                        const uint32_t wg = wi ? w0.y : w0.x;
+                        const uint32_t wg8 = wi ? w1.y : w1.x;
+                        uint32_t a[4];
+                        a[0] = lds32(lut + lut_off(wg, j0));
+                        a[1] = lds32(lut + lut_off(wg8, j0));
+                        a[2] = lds32(lut + lut_off(wg, j1));
+                        a[3] = lds32(lut + lut_off(wg8, j1));
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) Mma<D>::run(blk[nt], a, xf[s4][nt].x, xf[s4][nt].y);
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            acc[mt][nt][i] = __fmaf_rn(blk[nt][i], (i >> 1) ? a1 : a0, acc[mt][nt][i]);
+                }
             }
-        };
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.empty[st]);  // one arrival per warp, after all its reads
+        }
+    }
 
-        float acc[MT][NT][4];
+    // ----------------- output: stage the sums, add the cluster's partials
+    // (S > 1) and store.  Every thread of every CTA of the cluster passes the
+    // same barriers.  The ring is idle: every stage was consumed or drained.
+    __syncthreads();
+    float *stg = reinterpret_cast<float *>(&s.w[0][0]);  // [kRowsMax][NTOK]
+    if (warp >= 1) {
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) acc[mt][nt][i] = 0.f;
-
-        Frag cur, nxt;
-        uint2 xc[4][NT], xn[4][NT];
-        if (b_lo < b_hi) {
-            fetch(b_lo, cur);
-            fetch_x(b_lo, xc);
-        }
-        for (int b = b_lo; b < b_hi; ++b) {
-            if (b + 1 < b_hi) {
-                fetch(b + 1, nxt);
-                fetch_x(b + 1, xn);
-            }
-            float blk[MT][NT][4];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) blk[mt][nt][i] = 0.f;
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const int wi = s >> 1, j0 = 2 * (s & 1), j1 = j0 + 1;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const uint32_t wg = wi ? cur.w[mt][0].y : cur.w[mt][0].x;
-                    const uint32_t wg8 = wi ? cur.w[mt][1].y : cur.w[mt][1].x;
-                    uint32_t a[4];
-                    a[0] = lds32(lut_base + lut_off(wg, j0, lane4));
-                    a[1] = lds32(lut_base + lut_off(wg8, j0, lane4));
-                    a[2] = lds32(lut_base + lut_off(wg, j1, lane4));
-                    a[3] = lds32(lut_base + lut_off(wg8, j1, lane4));
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) Mma<D>::run(blk[mt][nt], a, xc[s][nt].x, xc[s][nt].y);
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = 16 * (wc + NCW * mt) + g + 8 * (i >> 1);
+                    stg[rr * NTOK + nt * 8 + 2 * t + (i & 1)] = acc[mt][nt][i];
                 }
-            }
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        acc[mt][nt][i] = __fmaf_rn(blk[mt][nt][i], cur.a[mt][i >> 1], acc[mt][nt][i]);
-            cur = nxt;
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) xc[s][nt] = xn[s][nt];
-        }
-
-        // this warp's partial sums -> shared sums (warps of a group split K)
-        if (active) {
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int tile = gi * MT + mt;
-                if (tile >= T) continue;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = 16 * tile + 8 * (i >> 1) + g;
-                        const int m = nt * 8 + 2 * t + (i & 1);
-                        if (m < M) atomicAdd(&sum[r * kMaxM + m], acc[mt][nt][i]);
-                    }
-            }
-        }
     }
-    __syncthreads();
-    for (int e = tid; e < T * 16 * kMaxM; e += kThreads) {
-        const int r = e / kMaxM, m = e % kMaxM;
-        const int row = r0 + r;
-        if (m < M && row < r1) {
-            float v = sum[e];
-            if (bias) v += Dt<D>::to_f32(bias[row]);
-            Y[(int64_t)m * N + row] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);
+    if (S > 1) cluster_sync_all();
+    else __syncthreads();
+    const uint32_t stg_addr = smem_u32(stg);
+    const int q_lo = (int)(((int64_t)R * z) / S), q_hi = (int)(((int64_t)R * (z + 1)) / S);
+    const int nr = q_hi - q_lo;
+    for (int v = threadIdx.x; v < nr * NT * 8; v += THREADS) {
+        const int m = v / nr, lr = q_lo + v % nr;  // consecutive threads: consecutive rows
+        if (m >= M) continue;
+        float sum;
+        if (S > 1) {
+            float p[8];
+            const uint32_t la = stg_addr + (uint32_t)(lr * NTOK + m) * 4;
+#pragma unroll
+            for (int q2 = 0; q2 < 8; ++q2)
+                if (q2 < S) p[q2] = ld_dsmem_f32(la, (uint32_t)q2);
+            sum = p[0];
+#pragma unroll
+            for (int q2 = 1; q2 < 8; ++q2)
+                if (q2 < S) sum += p[q2];
+        } else {
+            sum = stg[lr * NTOK + m];
         }
+        const int row = r0 + lr;
+        if (bias) sum += Dt<D>::to_f32(bias[row]);
+        Y[(int64_t)m * N + row] = (uint16_t)(Dt<D>::pack2(sum, 0.f) & 0xffffu);
     }
+    if (S > 1) cluster_sync_all();
 }
 
-size_t smem_bytes(int tiles) { return 256 * 32 * 4 + (size_t)tiles * 16 * kMaxM * 4; }
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 template <typename D, int NT>
-cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const void *bias,
-                     void *Y, int M, int N, int K, int log2B, const CodeTable &tab,
-                     cudaStream_t stream) {
-    const int G = device_sm_count();
-    const int max_rows = (N + G - 1) / G;
-    const int tiles = (max_rows + 15) / 16;
-    if (tiles > kMaxTiles) return cudaErrorInvalidValue;
-    const size_t smem = smem_bytes(tiles);
-    static int smem_set = 0;  // largest dynamic shared memory size set so far
-    if ((int)smem > 48 * 1024 && (int)smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_small_kernel<D, NT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        smem_set = (int)smem;
+cudaError_t set_smem_attr() {
+    static std::atomic<bool> done{false};
+    if (done.load(std::memory_order_relaxed)) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(gemm_small_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e == cudaSuccess) done.store(true, std::memory_order_relaxed);
+    return e;
+}
+
+cudaLaunchConfig_t make_cfg(dim3 grid, int S, cudaStream_t stream, cudaLaunchAttribute *attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = S;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+// CTAs in clusters of S (1, 2, 4, 8) resident at once on the current device
+template <typename D, int NT>
+int cluster_capacity(int S) {
+    static std::atomic<int> cache[64][4];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    const int si = S == 1 ? 0 : S == 2 ? 1 : S == 4 ? 2 : 3;
+    int v = cache[dev][si].load(std::memory_order_relaxed);
+    if (v == 0) {
+        int n = 0;
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = make_cfg(dim3(1, 1, S), S, 0, attr);
+        if (set_smem_attr<D, NT>() != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, gemm_small_kernel<D, NT>, &cfg) != cudaSuccess || n <= 0) {
+            (void)cudaGetLastError();
+            n = device_sm_count() / S;
+        }
+        v = n * S;
+        cache[dev][si].store(v, std::memory_order_relaxed);
     }
-    gemm_small_kernel<D, NT><<<G, kThreads, smem, stream>>>(
-        static_cast<const uint16_t *>(X), W, absmax, static_cast<const uint16_t *>(bias),
-        static_cast<uint16_t *>(Y), M, N, K, log2B, tab);
-    return cudaGetLastError();
+    return v;
+}
+
+// Row groups G and K split S.  A CTA's time is taken as its runs times
+// max(rows, 64) (fewer rows leave compute warps idle), plus a fixed cost per
+// split for the reduction.
+struct Plan {
+    int G, S;
+};
+
+template <typename D, int NT>
+Plan make_plan(int N, int nb) {
+    Plan best{1, 1};
+    double best_t = 1e300;
+    const int nq = (nb + RPS - 1) / RPS;  // stages of RPS runs; a split takes whole stages
+    for (int S = 1; S <= 8 && S <= nq; S *= 2) {
+        const int cap = cluster_capacity<D, NT>(S);
+        long G = cap / S;
+        if (G > (N + 15) / 16) G = (N + 15) / 16;  // at least 16 rows per group
+        if (G < 1) G = 1;
+        if ((N + G - 1) / G > kRowsMax) G = (N + kRowsMax - 1) / kRowsMax;
+        const long rows = (N + G - 1) / G;
+        const long waves = (G * S + cap - 1) / cap;
+        const double t = (double)waves * (RPS * ((nq + S - 1) / S) * (double)(rows > 64 ? rows : 64) +
+                                          (S > 1 ? 4.0 * 64 : 0.0));
+        if (t < best_t - 1e-9) {
+            best_t = t;
+            best = Plan{(int)G, S};
+        }
+    }
+    return best;
+}
+
+template <typename D, int NT>
+cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const void *bias, void *Y,
+                     int M, int N, int K, int log2B, const CodeTable &tab, cudaStream_t stream) {
+    if (!get_encode()) return cudaErrorNotSupported;
+    const int nb = K / RUN;
+    const Plan plan = make_plan<D, NT>(N, nb);
+    const int rbox = (N + plan.G - 1) / plan.G;
+    const CUtensorMapDataType xt = std::is_same<D, BF16>::value ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                                : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUtensorMap map_w, map_x, map_amx;
+    const uint64_t row_bytes = (uint64_t)K / 2;
+    if (encode_2d(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, W, row_bytes, N, row_bytes, RPS * RUN / 2, rbox,
+                  CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+        encode_2d(&map_x, xt, X, K, M, (uint64_t)K * 2, RUN, NTOK, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const int nblk = K >> log2B;
+    int amx_tma = nblk % 4 == 0 ? 1 : 0;
+    std::memset(&map_amx, 0, sizeof(map_amx));
+    if (amx_tma && encode_2d(&map_amx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, absmax, nblk, N, (uint64_t)nblk * 4, 4,
+                             rbox, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+        amx_tma = 0;
+    cudaError_t e = set_smem_attr<D, NT>();
+    if (e != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = make_cfg(dim3(plan.G, 1, plan.S), plan.S, stream, attr);
+    return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT>, map_w, map_amx, map_x, absmax,
+                              static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(Y), M, N, K,
+                              log2B, amx_tma, rbox, tab);
 }
 
 }  // namespace

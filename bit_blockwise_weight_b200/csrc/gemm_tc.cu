@@ -40,19 +40,15 @@
 // Every mbarrier wait is bounded (about one second of %globaltimer); a wait
 // that runs out raises the library's device error word, makes the CTA skip
 // the rest of its work, and still frees its TMEM before returning.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <atomic>
 #include <cstring>
 #include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace bnb4 {
-
-__device__ unsigned int g_device_error = 0;  // raised by a timed-out wait
 
 namespace {
 
@@ -72,7 +68,6 @@ constexpr int RED_PITCH = RED_CW + 4;            // fp32 staging row pitch
 constexpr int NUM_DQ_WARPS = 8;
 constexpr int W_WARP = 2 + NUM_DQ_WARPS;          // weight-tile producer
 constexpr int THREADS = (3 + NUM_DQ_WARPS) * 32;  // 352
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // ~1 s
 
 struct Smem {
     uint8_t a[A_STAGES][A_STAGE];   // 1024-byte aligned (swizzle atoms)
@@ -88,156 +83,6 @@ struct Smem {
 };
 static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory plan");
 static_assert(BM * RED_PITCH * 4 <= A_STAGES * A_STAGE, "split-K staging fits in the A ring");
-
-// ------------------------------------------------------------------ PTX
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Bounded wait: false (and the error word raised, the CTA told to abort) when
-// the barrier did not reach the phase within the limit or another thread of
-// the CTA already gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicAdd(&g_device_error, 1u);
-            return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(const CUtensorMap *map, uint64_t *bar, void *dst,
-                                            int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_ld_wait() {
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle, sm100 version 1.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3fff);
-    d |= (uint64_t)((lbo_bytes >> 4) & 0x3fff) << 16;
-    d |= (uint64_t)((sbo_bytes >> 4) & 0x3fff) << 32;
-    d |= (uint64_t)1 << 46;  // version
-    d |= (uint64_t)2 << 61;  // SWIZZLE_128B
-    return d;
-}
-
-// Instruction descriptor for kind::f16: fp32 accumulate, M = 128, N = BN.
-template <int BN>
-__host__ __device__ constexpr uint32_t make_idesc(bool bf16, bool b_mn_major) {
-    return (1u << 4)                              // D format: F32
-           | ((bf16 ? 1u : 0u) << 7)              // A format
-           | ((bf16 ? 1u : 0u) << 10)             // B format
-           | ((b_mn_major ? 1u : 0u) << 16)       // B major (A is K-major)
-           | ((uint32_t)(BN >> 3) << 17)          // N
-           | ((uint32_t)(128 >> 4) << 24);        // M
-}
-
-// Byte offset of the 16-byte chunk j of 128-byte row `row` inside a
-// 128-byte-swizzled region whose 8-row atoms sit `atom_stride` apart:
-// physical chunk = j ^ (row mod 8).
-__device__ __forceinline__ uint32_t swz(uint32_t row_base, uint32_t row, uint32_t j) {
-    return row_base + ((j ^ (row & 7u)) << 4);
-}
-
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                     : "memory");
-}
-
-__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t local_addr, uint32_t rank) {
-    uint32_t remote;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(remote)
-                 : "memory");
-    return v;
-}
 
 template <typename D, int CNT>
 __device__ __forceinline__ void store_out(uint16_t *out, int64_t row, int n_out, int col,
@@ -269,17 +114,6 @@ __device__ __forceinline__ void store_out(uint16_t *out, int64_t row, int n_out,
         for (int e = 0; e < CNT; ++e)
             if (col + e < n_out) dst[e] = (uint16_t)(Dt<D>::pack2(w[e], 0.f) & 0xffffu);
     }
-}
-
-// Bounded wait used before a CTA exits: lets loads still in flight land in its
-// shared memory even when the CTA is aborting.
-__device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > kWaitLimitNs) {
-            atomicAdd(&g_device_error, 1u);
-            return;
-        }
 }
 
 template <typename D, bool BWD, int BN>
@@ -414,7 +248,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc<BN>(std::is_same<D, BF16>::value, BWD);
+            constexpr uint32_t idesc = make_idesc<BN, 128>(std::is_same<D, BF16>::value, BWD);
             bool ok = true;
             for (int i = 0; i < iters && ok; ++i) {
                 const int sa = i % A_STAGES, sb = i % B_STAGES;
@@ -619,19 +453,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *p = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 template <typename D, bool BWD, int BN>
@@ -726,18 +547,6 @@ Plan make_plan(long mt, int n_out, int iters) {
         }
     }
     return best;
-}
-
-CUresult encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t inner,
-                   uint64_t outer, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer,
-                   CUtensorMapSwizzle swizzle) {
-    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-    cuuint64_t strides[1] = {(cuuint64_t)pitch_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    return get_encode()(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 template <typename D, bool BWD>

@@ -27,7 +27,7 @@ cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, co
                         void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
                         bnb4_dtype dt, cudaStream_t stream);
 
-// 1 <= M <= 16: weights decoded in registers into mma.sync fragments
+// 1 <= M <= 16: weights decoded into tensor memory, tcgen05.mma with N = 16 tokens
 cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
                               const void *bias, void *Y, int64_t M, int64_t N, int64_t K,
                               int blocksize, bnb4_quant_type qt, bnb4_dtype dt,

@@ -4,7 +4,8 @@ Two layers, both argument marshalling only (every step of the computation
 runs in the library's CUDA kernels):
 
 * ``bnb4_quantize``, ``bnb4_dequantize``, ``bnb4_gemv``, ``bnb4_gemm``,
-  ``bnb4_gemm_backward``: the C ABI of ``include/bnb4.h`` one to one (raw
+  ``bnb4_gemm_backward``, ``bnb4_device_status``,
+  ``bnb4_selftest_wait_timeout``: the C ABI of ``include/bnb4.h`` one to one (raw
   device pointers as ints, sizes, enums, a ``cudaStream_t`` as an int).
   They return the integer status.
 * ``quantize_4bit``, ``dequantize_4bit``, ``gemv_4bit``, ``gemm_4bit``,
@@ -50,6 +51,8 @@ def _load() -> ctypes.CDLL:
         "bnb4_gemv": (I, [P, P, P, P, P, I64, I64, I, I, I, P]),
         "bnb4_gemm": (I, [P, P, P, P, P, I64, I64, I64, I, I, I, P]),
         "bnb4_gemm_backward": (I, [P, P, P, P, I64, I64, I64, I, I, I, P]),
+        "bnb4_device_status": (I, [P]),
+        "bnb4_selftest_wait_timeout": (I, [P]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(L, name)
@@ -67,6 +70,8 @@ bnb4_dequantize = _lib.bnb4_dequantize
 bnb4_gemv = _lib.bnb4_gemv
 bnb4_gemm = _lib.bnb4_gemm
 bnb4_gemm_backward = _lib.bnb4_gemm_backward
+bnb4_device_status = _lib.bnb4_device_status
+bnb4_selftest_wait_timeout = _lib.bnb4_selftest_wait_timeout
 
 
 def status_string(status: int) -> str:
@@ -185,3 +190,9 @@ def gemm_4bit_backward(dY, packed, absmax, K: int, blocksize: int = 64, quant_ty
                               _qtype(quant_type), _dtype_code(dY), _stream(stream)),
            "bnb4_gemm_backward")
     return dX
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the count of bounded device
+    waits that gave up: STATUS_OK, or the BNB4_ERR_TIMEOUT / BNB4_ERR_CUDA code."""
+    return int(bnb4_device_status(_stream(stream)))

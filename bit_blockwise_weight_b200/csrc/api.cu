@@ -136,4 +136,16 @@ bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *ab
     return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true, stream));
 }
 
+bnb4_status bnb4_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return BNB4_ERR_CUDA;
+    unsigned int a = 0, b = 0;
+    if (gemm_tc_take_timeouts(&a) != cudaSuccess || gemm_small_take_timeouts(&b) != cudaSuccess)
+        return BNB4_ERR_CUDA;
+    return (a != 0 || b != 0) ? BNB4_ERR_TIMEOUT : BNB4_OK;
+}
+
+bnb4_status bnb4_selftest_wait_timeout(cudaStream_t stream) {
+    return from_cuda(launch_selftest_wait_timeout(stream));
+}
+
 }  // extern "C"

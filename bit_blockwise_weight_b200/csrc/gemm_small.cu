@@ -417,6 +417,8 @@ cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const
 
 }  // namespace
 
+cudaError_t gemm_small_take_timeouts(unsigned int *count) { return take_wait_timeouts(count); }
+
 cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
                               const void *bias, void *Y, int64_t M, int64_t N, int64_t K,
                               int blocksize, bnb4_quant_type qt, bnb4_dtype dt,

@@ -597,7 +597,28 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
                                   tab, C, stream);
 }
 
+// A wait that nothing completes, bounded at limit_ns: exercises the timeout
+// path (error count raised, no fault, the kernel returns).
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_wait_timeout(cudaStream_t stream) {
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(1000000ull);  // 1 ms
+    return cudaGetLastError();
+}
+
+cudaError_t gemm_tc_take_timeouts(unsigned int *count) { return take_wait_timeouts(count); }
 
 cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax, const void *bias,
                            void *D, int64_t M, int64_t N, int64_t K, int blocksize,

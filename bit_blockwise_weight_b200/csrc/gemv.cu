@@ -27,8 +27,7 @@
 //   * when a warp leaves a quad, its 4 row sums are reduced across lanes with
 //     xor-shuffles and added to the CTA's row sums in shared memory.
 // The codes enter as 16-bit values (the code table rounded once to bf16 /
-// fp16), like the weight operand of the tensor-core kernels.  No global
-// scratch.
+// fp16), as in the small-M kernel.  No global scratch.
 #include "common.cuh"
 #include "kernels.h"
 

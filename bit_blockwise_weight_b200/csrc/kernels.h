@@ -40,6 +40,13 @@ cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax,
                            int blocksize, bnb4_quant_type qt, bnb4_dtype dt, bool backward,
                            cudaStream_t stream);
 
+// read and clear the count of bounded waits that gave up, per kernel file
+cudaError_t gemm_tc_take_timeouts(unsigned int *count);
+cudaError_t gemm_small_take_timeouts(unsigned int *count);
+
+// one kernel whose mbarrier wait runs out after 1 ms (tests the timeout path)
+cudaError_t launch_selftest_wait_timeout(cudaStream_t stream);
+
 // largest M handled by launch_gemm_small
 constexpr int64_t kSmallMMax = 16;
 

@@ -58,13 +58,14 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Bounded wait: false (and the error word raised, the CTA told to abort) when
 // the barrier did not reach the phase within the limit or another thread of
 // the CTA already gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
             *abort = 1;
             atomicAdd(&g_wait_timeouts, 1u);
             return false;
@@ -233,6 +234,15 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------ host side
+
+// Read and clear this file's count of timed-out waits on the current device.
+inline cudaError_t take_wait_timeouts(unsigned int *count) {
+    cudaError_t e = cudaMemcpyFromSymbol(count, g_wait_timeouts, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(unsigned int));
+}
+
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;

@@ -31,10 +31,15 @@
  *     nibble); an odd last element leaves the low nibble 0.
  *   - dequantized value = RN_dtype(fp32(code[idx] * absmax)): one fp32
  *     product, then one round-to-nearest-even conversion.
- *   - matmuls accumulate in fp32.  They consume the weight dequantized as
- *     above and rounded to the compute dtype (bf16 / fp16); the result is
- *     rounded once to the compute dtype.  The bias, if given, is added in
- *     fp32 before that rounding.
+ *   - matmuls accumulate in fp32 and round the result once to the compute
+ *     dtype (bf16 / fp16); the bias, if given, is added in fp32 before that
+ *     rounding.  For M >= 17 and the backward the weight is the dequantized
+ *     value above (already in the compute dtype).  For M <= 16 (gemv
+ *     included) each code is rounded to the compute dtype and the fp32 sums
+ *     are scaled by the block's absmax: the same weight up to one rounding of
+ *     the code (2^-9 relative in bf16, 2^-12 in fp16).  Either way the result
+ *     stays within 5e-3 relative L2 of the float64 product with the
+ *     dequantized weights.
  *
  * Weight layout for the matmuls: W is [N, K] row-major (out x in, like a
  * Linear layer's weight) and was quantized as one flat array of N*K
@@ -141,13 +146,36 @@ bnb4_status bnb4_gemm(const void *X, const uint8_t *packedW,
  * Backward of bnb4_gemm with respect to its input:
  *   dX[M, K] = dY[M, N] @ dequant(W)   (reduction over N, no bias term).
  *   dY [M, N] of dt;  dX [M, K] of dt (out); same weight arguments and
- *   constraints as bnb4_gemm.
+ *   constraints as bnb4_gemm, plus N % 8 == 0 (dY rows are read with TMA,
+ *   which needs a 16-byte row pitch).
  */
 bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *packedW,
                                const float *absmax, void *dX, int64_t M,
                                int64_t N, int64_t K, int blocksize,
                                bnb4_quant_type quant_type, bnb4_dtype dt,
                                cudaStream_t stream);
+
+/*
+ * Device-side status of the library's kernels (no counterpart on the pages:
+ * a diagnostic for the bounded waits of the tensor-core kernels).  Every
+ * mbarrier wait in those kernels gives up after about one second; a kernel
+ * whose wait gave up skips its remaining work (its outputs are then
+ * undefined), frees its tensor memory and returns.
+ * Synchronises `stream` (blocking the host), then reads and clears the
+ * count of waits that gave up on the current device since the last call.
+ * Returns BNB4_ERR_TIMEOUT if any did, BNB4_ERR_CUDA if the synchronisation
+ * or the read failed (for instance after an earlier launch error), else
+ * BNB4_OK.
+ */
+bnb4_status bnb4_device_status(cudaStream_t stream);
+
+/*
+ * Enqueues one small kernel whose mbarrier wait nothing completes; the wait
+ * gives up after 1 ms, so the next bnb4_device_status reports
+ * BNB4_ERR_TIMEOUT.  For testing the timeout path without faulting or
+ * hanging the GPU.
+ */
+bnb4_status bnb4_selftest_wait_timeout(cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -40,7 +40,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"libbnb4.so not found at {LIB_PATH}; build it with "
-            "`python -m bit_blockwise_weight_b200.build` (needs nvcc)")
+            "`python bit_blockwise_weight_b200/build.py` (needs nvcc)")
     L = ctypes.CDLL(LIB_PATH)
     P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     sigs = {

@@ -1,6 +1,7 @@
 """Build libbnb4.so in-tree from csrc/*.cu with nvcc for sm_100a.
 
-Usage: python -m bit_blockwise_weight_b200.build [--force]
+Usage: python bit_blockwise_weight_b200/build.py [--force]  (run as a file: importing the
+package loads the library this builds)
 """
 from __future__ import annotations
 

@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
             "oracle_matmul_entries": (I, [P, I, P, P, P, I64, I64, I64, I, I, P, P, I64, P]),
             "oracle_matmul_backward": (I, [P, I, P, P, I64, I64, I64, I, I, P]),
             "oracle_matmul_backward_entries": (I, [P, I, P, P, I64, I64, I64, I, I, P, P, I64, P]),
+            "oracle_double_quant": (I, [P, I64, I, P, P]),
+            "oracle_dequant_absmax": (I, [P, P, I64, I, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -186,3 +188,27 @@ def matmul_backward_entries(dY, dy_dtype, packed, absmax, M, N, K, blocksize, qt
                                                 QTYPES[qtype], _ptr(ms), _ptr(ks), ms.size,
                                                 _ptr(dX)), "matmul_backward_entries")
     return dX
+
+
+def double_quant(absmax, group=256):
+    """R9: (q uint8 [n], scales float32 [ceil(n / group)]) of an fp32 absmax array."""
+    absmax = np.ascontiguousarray(absmax, np.float32).reshape(-1)
+    if group < 1:
+        raise ValueError("group must be >= 1")
+    q = np.empty(absmax.size, np.uint8)
+    scales = np.empty((absmax.size + group - 1) // group, np.float32)
+    _check(lib().oracle_double_quant(_ptr(absmax), absmax.size, group, _ptr(q), _ptr(scales)),
+           "double_quant")
+    return q, scales
+
+
+def dequant_absmax(q, scales, group=256):
+    """R9 inverse: fp32(q) * fp32(scale / 255)."""
+    q = np.ascontiguousarray(q, np.uint8).reshape(-1)
+    scales = np.ascontiguousarray(scales, np.float32).reshape(-1)
+    if group < 1 or scales.size != (q.size + group - 1) // group:
+        raise ValueError("scales must hold one value per group")
+    out = np.empty(q.size, np.float32)
+    _check(lib().oracle_dequant_absmax(_ptr(q), _ptr(scales), q.size, group, _ptr(out)),
+           "dequant_absmax")
+    return out

@@ -372,3 +372,44 @@ int oracle_matmul_backward_entries(const void *dY, int dy_dtype,
     }
     return 0;
 }
+
+/* ------------------------------------------------ double quantization (R9) */
+
+int oracle_double_quant(const float *absmax, int64_t n, int group, uint8_t *q,
+                        float *scales)
+{
+    if (group < 1 || n < 0)
+        return -1;
+    for (int64_t g0 = 0; g0 < n; g0 += group) {
+        const int64_t g1 = g0 + group < n ? g0 + group : n;
+        float s = 0.0f;
+        for (int64_t i = g0; i < g1; ++i)
+            if (absmax[i] > s)
+                s = absmax[i];
+        scales[g0 / group] = s;
+        for (int64_t i = g0; i < g1; ++i) {
+            uint8_t code = 0;
+            if (s > 0.0f) {
+                const float v = absmax[i] / s;  /* fp32 quotient */
+                const float t = v * 255.0f;     /* fp32 product */
+                const float r = rintf(t);       /* ties to even */
+                if (r > 0.0f)                   /* NaN and r <= 0 give 0 */
+                    code = r >= 255.0f ? (uint8_t)255 : (uint8_t)r;
+            }
+            q[i] = code;
+        }
+    }
+    return 0;
+}
+
+int oracle_dequant_absmax(const uint8_t *q, const float *scales, int64_t n,
+                          int group, float *out)
+{
+    if (group < 1 || n < 0)
+        return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        const float step = scales[i / group] / 255.0f;  /* fp32 quotient */
+        out[i] = (float)q[i] * step;                    /* fp32 product */
+    }
+    return 0;
+}

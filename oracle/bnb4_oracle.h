@@ -16,6 +16,9 @@
  *     quantize_4bit, dequantize_4bit, gemv_4bit, gemm_4bit,
  *     gemm_4bit_backward = grad_output @ dequantize_4bit(B)) and section
  *     "Correctness" (exact nearest-code search, never through a lookup table).
+ *   - "mps-bitsandbytes 0.4.7", Functional API, Double Quantization
+ *     (double_quant(absmax, double_quant_block=256) -> (absmax_quant,
+ *     absmax_scales); dequant_absmax restores the scales).
  */
 #ifndef BNB4_ORACLE_H
 #define BNB4_ORACLE_H
@@ -81,6 +84,22 @@ int oracle_matmul_backward_entries(const void *dY, int dy_dtype,
                                    int64_t M, int64_t N, int64_t K,
                                    int blocksize, int qtype, const int64_t *ms,
                                    const int64_t *ks, int64_t count, double *dX);
+
+/* R9 -- double quantization of an absmax array (the pages give only the
+ * call and the group of 256; this is the plainest reading).  Groups of
+ * `group` consecutive values (the last one may be short):
+ *   scale[g] = max over the group of absmax[i] (values that are not > the
+ *              running maximum, NaN included, are skipped; +0 if none is > 0);
+ *   q[i]     = clamp(rint(fp32(fp32(absmax[i] / scale[g]) * 255)), 0, 255),
+ *              rint rounding ties to even, NaN -> 0, and 0 when scale[g] == 0;
+ * and the inverse
+ *   out[i]   = fp32(q[i]) * fp32(scale[g] / 255)   (each step one fp32 rounding).
+ * An unsigned linear 8-bit code: absmax values are >= 0.
+ * Return 0, or -1 when group < 1 or n < 0. */
+int oracle_double_quant(const float *absmax, int64_t n, int group, uint8_t *q,
+                        float *scales);
+int oracle_dequant_absmax(const uint8_t *q, const float *scales, int64_t n,
+                          int group, float *out);
 
 #ifdef __cplusplus
 }

@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 import test_oracle as pins  # noqa: E402  (tests/ is on sys.path under pytest)
+import test_oracle_double_quant as dq_pins  # noqa: E402
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "bnb4_oracle.c")
 
@@ -42,6 +43,11 @@ MUTATIONS = {
     "forward_bias_dropped": ("acc += (double)load_elem(bias, x_dtype, j);", "acc += 0.0;"),
     "backward_weight_transposed": ("j * K + k, blocksize, code);\n        acc += g * wv;",
                                    "k * N + j, blocksize, code);\n        acc += g * wv;"),
+    "double_quant_truncates": ("const float r = rintf(t);", "const float r = truncf(t);"),
+    "double_quant_scale_is_first_value": ("if (absmax[i] > s)\n                s = absmax[i];",
+                                          "if (i == g0)\n                s = absmax[i];"),
+    "dequant_absmax_other_rounding_order": ("out[i] = (float)q[i] * step;",
+                                            "out[i] = (float)q[i] * scales[i / group] / 255.0f;"),
 }
 
 PIN_CHECKS = [
@@ -57,6 +63,9 @@ PIN_CHECKS = [
     lambda: pins.test_f32_to_16bit_rne_against_torch_and_numpy(),
     lambda: pins.test_matmul_one_hot_gives_weight_column(),
     lambda: [pins.test_matmul_and_backward_exact_bruteforce(q) for q in ("nf4",)],
+    lambda: [dq_pins.test_double_quant_matches_exact_rationals(g) for g in (4, 7, 256)],
+    lambda: dq_pins.test_double_quant_closed_forms(),
+    lambda: dq_pins.test_double_quant_special_values(),
 ]
 
 
@@ -85,7 +94,8 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
         for attr in ("oracle_code_table", "oracle_to_f32_array", "oracle_from_f32_array",
                      "oracle_quantize", "oracle_dequantize", "oracle_matmul",
                      "oracle_matmul_entries", "oracle_matmul_backward",
-                     "oracle_matmul_backward_entries"):
+                     "oracle_matmul_backward_entries", "oracle_double_quant",
+                     "oracle_dequant_absmax"):
             f, g = getattr(real, attr), getattr(mutant, attr)
             g.restype, g.argtypes = f.restype, f.argtypes
         monkeypatch.setattr(oracle, "_lib", mutant)

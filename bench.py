@@ -289,6 +289,9 @@ def run_ours(args, rank, world, dev):
     step_bytes = sum(b for _, b, _ in ops)
     value = step_bytes * args.steps * world / (ms / 1e3) / 1e9
 
+    # the next rows beyond the step (double-quantized statistics), timed on their own
+    next_rows = time_next_rows(step, dev, args.steps, hbm)
+
     # e2e: the same step through the public API from pinned host buffers; the step's
     # inputs go host->device and every output comes back device->host, every step
     e2e = run_e2e(args, step, dev, stream)
@@ -334,6 +337,7 @@ def run_ours(args, rank, world, dev):
                              "event node after each launch"},
         "roofline": roof,
         "parts": parts,
+        "next_rows": next_rows,
         "e2e": e2e,
         "gpu_launches": len(calls) * args.steps,
         "clocks": clocks,
@@ -342,6 +346,70 @@ def run_ours(args, rank, world, dev):
     if args.cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     return line
+
+
+def time_next_rows(step, dev, steps, hbm):
+    """Double quantization of absmax and the gemv on 8-bit statistics, outside
+    the step: double_quant / dequant_absmax on the step's absmax (2^22 values,
+    groups of 256), and each gemv shape with fp32 absmax and with its
+    double-quantized absmax, side by side.  L2 is flushed (a 512 MB fill)
+    before every op; one CUDA graph holds flush, event, op, event per op."""
+    b = step.bnb4
+    G = 256
+    n = step.absmax.numel()
+    aq = torch.empty(n, dtype=torch.uint8, device=dev)
+    asc = torch.empty((n + G - 1) // G, dtype=torch.float32, device=dev)
+    back = torch.empty(n, dtype=torch.float32, device=dev)
+    b.double_quant(step.absmax, G, out=(aq, asc))
+    ops = [("double_quant_absmax_4194304", 4 * n + n + 4 * asc.numel(),
+            lambda: b.double_quant(step.absmax, G, out=(aq, asc))),
+           ("dequant_absmax_4194304", n + 4 * asc.numel() + 4 * n,
+            lambda: b.dequant_absmax(aq, asc, G, out=back))]
+    for K, N, p, a, xv, bias, y in step.gemv:
+        q8, s8 = b.double_quant(a, G)
+        nb = N * K // BLOCK
+        ops.append((f"gemv_4bit_{K}x{N}", N * K // 2 + 4 * nb + 2 * K + 4 * N,
+                    lambda K=K, N=N, p=p, a=a, xv=xv, bias=bias, y=y:
+                    b.gemv_4bit(xv, p, a, N, K, bias, BLOCK, "nf4", out=y)))
+        ops.append((f"gemv_4bit_dq_{K}x{N}", N * K // 2 + nb + 4 * s8.numel() + 2 * K + 4 * N,
+                    lambda K=K, N=N, p=p, q8=q8, s8=s8, xv=xv, bias=bias, y=y:
+                    b.gemv_4bit_dq(xv, p, q8, s8, N, K, bias, BLOCK, "nf4", G, out=y)))
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in ops]
+    for _, _, f in ops:
+        f()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for (_, _, f), (e0, e1) in zip(ops, ev):
+            flush.fill_(1)
+            e0.record(cap)
+            f()
+            e1.record(cap)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    times = [[] for _ in ops]
+    for _ in range(max(3, min(steps, 20))):
+        g.replay()
+        torch.cuda.synchronize(dev)
+        for i, (e0, e1) in enumerate(ev):
+            times[i].append(e0.elapsed_time(e1))
+    del g
+    out = {}
+    for (nm, nbytes, _), t in zip(ops, times):
+        us = statistics.median(t) * 1e3
+        gbs = nbytes / (us / 1e6) / 1e9
+        out[nm] = {"us": round(us, 2), "bytes": nbytes, "GB/s": round(gbs, 1),
+                   "hbm_frac": round(gbs / hbm, 4)}
+    for K, N, *_ in step.gemv:
+        out[f"gemv_4bit_dq_{K}x{N}"]["speedup_vs_fp32_absmax"] = round(
+            out[f"gemv_4bit_{K}x{N}"]["us"] / out[f"gemv_4bit_dq_{K}x{N}"]["us"], 3)
+    out["note"] = ("L2 flushed before each op; median of the replays; each time includes the "
+                   "few us of its two event nodes")
+    return out
 
 
 def run_e2e(args, step, dev, stream):
@@ -489,6 +557,9 @@ PROFILE_CASES = {
     "gemm_small": "gemm_4bit M=16, K=8192, N=28672, NF4 B=64, bf16",
     "gemm_tc": "gemm_4bit M=512, K=4096, N=14336, NF4 B=64, bf16",
     "gemm_tc_backward": "gemm_4bit_backward M=512, K=4096, N=14336, NF4 B=64, bf16",
+    "double_quant": "double_quant + dequant_absmax of 2^25 absmax values, groups of 256",
+    "gemv_dq": "gemv_4bit_dq + bias, K=4096, N=14336, NF4 B=64, double-quantized absmax "
+               "(groups of 256), bf16",
 }
 
 
@@ -507,8 +578,12 @@ def profile_case(name):
         p, a = bnb4.quantize_4bit(x, BLOCK, "nf4")
         if name == "dequantize":
             bnb4.dequantize_4bit(p, a, x.numel(), BLOCK, "nf4", dtype=torch.bfloat16)
+    elif name == "double_quant":
+        a = synthetic.absmax_values(1 << 25, seed=4).to(dev)
+        q, s = bnb4.double_quant(a, 256)
+        bnb4.dequant_absmax(q, s, 256)
     else:
-        K, N, M = {"gemv": (4096, 14336, 1), "gemm_small": (8192, 28672, 16),
+        K, N, M = {"gemv": (4096, 14336, 1), "gemv_dq": (4096, 14336, 1), "gemm_small": (8192, 28672, 16),
                    "gemm_tc": (4096, 14336, 512), "gemm_tc_backward": (4096, 14336, 512)}[name]
         w = synthetic.normal((N * K,), 0, 0.02, "f32", device=d)
         p, a = bnb4.quantize_4bit(w, BLOCK, "nf4")
@@ -516,6 +591,10 @@ def profile_case(name):
         if name == "gemv":
             bnb4.gemv_4bit(synthetic.normal((K,), 1, 1.0, "bf16", device=d), p, a, N, K,
                            synthetic.normal((N,), 2, 1.0, "bf16", device=d))
+        elif name == "gemv_dq":
+            q8, s8 = bnb4.double_quant(a, 256)
+            bnb4.gemv_4bit_dq(synthetic.normal((K,), 1, 1.0, "bf16", device=d), p, q8, s8, N, K,
+                              synthetic.normal((N,), 2, 1.0, "bf16", device=d))
         elif name == "gemm_tc_backward":
             bnb4.gemm_4bit_backward(synthetic.normal((M, N), 3, 1.0, "bf16", device=d), p, a, K)
         else:

@@ -4,8 +4,9 @@ Two layers, both argument marshalling only (every step of the computation
 runs in the library's CUDA kernels):
 
 * ``bnb4_quantize``, ``bnb4_dequantize``, ``bnb4_gemv``, ``bnb4_gemm``,
-  ``bnb4_gemm_backward``, ``bnb4_device_status``,
-  ``bnb4_selftest_wait_timeout``: the C ABI of ``include/bnb4.h`` one to one (raw
+  ``bnb4_gemm_backward``, ``bnb4_gemv_dq``, ``bnb4_double_quant``, ``bnb4_dequant_absmax``,
+  ``bnb4_device_status``, ``bnb4_selftest_wait_timeout``: the C ABI of
+  ``include/bnb4.h`` one to one (raw
   device pointers as ints, sizes, enums, a ``cudaStream_t`` as an int).
   They return the integer status.
 * ``quantize_4bit``, ``dequantize_4bit``, ``gemv_4bit``, ``gemm_4bit``,
@@ -51,6 +52,9 @@ def _load() -> ctypes.CDLL:
         "bnb4_gemv": (I, [P, P, P, P, P, I64, I64, I, I, I, P]),
         "bnb4_gemm": (I, [P, P, P, P, P, I64, I64, I64, I, I, I, P]),
         "bnb4_gemm_backward": (I, [P, P, P, P, I64, I64, I64, I, I, I, P]),
+        "bnb4_gemv_dq": (I, [P, P, P, P, I, P, P, I64, I64, I, I, I, P]),
+        "bnb4_double_quant": (I, [P, I64, I, P, P, P]),
+        "bnb4_dequant_absmax": (I, [P, P, I64, I, P, P]),
         "bnb4_device_status": (I, [P]),
         "bnb4_selftest_wait_timeout": (I, [P]),
     }
@@ -70,6 +74,9 @@ bnb4_dequantize = _lib.bnb4_dequantize
 bnb4_gemv = _lib.bnb4_gemv
 bnb4_gemm = _lib.bnb4_gemm
 bnb4_gemm_backward = _lib.bnb4_gemm_backward
+bnb4_gemv_dq = _lib.bnb4_gemv_dq
+bnb4_double_quant = _lib.bnb4_double_quant
+bnb4_dequant_absmax = _lib.bnb4_dequant_absmax
 bnb4_device_status = _lib.bnb4_device_status
 bnb4_selftest_wait_timeout = _lib.bnb4_selftest_wait_timeout
 
@@ -167,6 +174,18 @@ def gemv_4bit(x, packed, absmax, N: int, K: int, bias=None, blocksize: int = 64,
     return y
 
 
+def gemv_4bit_dq(x, packed, absmax_q, absmax_scales, N: int, K: int, bias=None,
+                 blocksize: int = 64, quant_type="nf4", group: int = 256, out=None, stream=None):
+    """gemv_4bit with the absmax given as double_quant's (codes, scales)."""
+    torch = _torch()
+    _need_cuda(x, packed, absmax_q, absmax_scales, bias)
+    y = out if out is not None else torch.empty(N, dtype=x.dtype, device=x.device)
+    _check(bnb4_gemv_dq(_ptr(x), _ptr(packed), _ptr(absmax_q), _ptr(absmax_scales), group, _ptr(bias),
+                        _ptr(y), N, K, blocksize, _qtype(quant_type), _dtype_code(x), _stream(stream)),
+           "bnb4_gemv_dq")
+    return y
+
+
 def gemm_4bit(X, packed, absmax, N: int, bias=None, blocksize: int = 64, quant_type="nf4",
               out=None, stream=None):
     """X [M, K] -> Y [M, N] = X @ dequant(W)^T (+ bias)."""
@@ -190,6 +209,40 @@ def gemm_4bit_backward(dY, packed, absmax, K: int, blocksize: int = 64, quant_ty
                               _qtype(quant_type), _dtype_code(dY), _stream(stream)),
            "bnb4_gemm_backward")
     return dX
+
+
+def double_quant(absmax, group: int = 256, out=None, stream=None):
+    """absmax float32 [n] (CUDA) -> (absmax_q uint8 [n], scales float32 [ceil(n/group)]);
+    out = (absmax_q, scales) writes into caller-provided buffers."""
+    torch = _torch()
+    _need_cuda(absmax)
+    if absmax.dtype != torch.float32:
+        raise TypeError("absmax must be float32")
+    n = absmax.numel()
+    if out is not None:
+        q, scales = out
+        _need_cuda(q, scales)
+        if q.numel() != n or scales.numel() != (n + group - 1) // group:
+            raise ValueError("out buffers have the wrong sizes")
+    else:
+        q = torch.empty(n, dtype=torch.uint8, device=absmax.device)
+        scales = torch.empty((n + group - 1) // group, dtype=torch.float32, device=absmax.device)
+    _check(bnb4_double_quant(_ptr(absmax), n, group, _ptr(q), _ptr(scales), _stream(stream)),
+           "bnb4_double_quant")
+    return q, scales
+
+
+def dequant_absmax(absmax_q, scales, group: int = 256, out=None, stream=None):
+    """Inverse of double_quant -> absmax float32 [n]."""
+    torch = _torch()
+    _need_cuda(absmax_q, scales)
+    n = absmax_q.numel()
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=absmax_q.device)
+    _need_cuda(out)
+    _check(bnb4_dequant_absmax(_ptr(absmax_q), _ptr(scales), n, group, _ptr(out), _stream(stream)),
+           "bnb4_dequant_absmax")
+    return out
 
 
 def device_status(stream=None) -> int:

@@ -110,10 +110,27 @@ bnb4_status bnb4_gemv(const void *x, const uint8_t *W, const float *absmax, cons
     bnb4_status s = check_matmul(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt);
     if (s != BNB4_OK) return s;
     if (N <= gemv_max_rows() && K <= gemv_max_k())
-        return from_cuda(launch_gemv(x, W, absmax, bias, y, N, K, blocksize, qt, dt, stream));
+        return from_cuda(launch_gemv(x, W, absmax, nullptr, nullptr, 0, bias, y, N, K, blocksize, qt, dt,
+                                     stream));
     // shapes beyond the CUDA-core kernel's shared-memory plan: the same product
     // through the matrix kernels (x is a 1 x K matrix)
     return bnb4_gemm(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt, stream);
+}
+
+bnb4_status bnb4_gemv_dq(const void *x, const uint8_t *W, const uint8_t *absmax_q,
+                         const float *absmax_scales, int group, const void *bias, void *y, int64_t N,
+                         int64_t K, int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+                         cudaStream_t stream) {
+    if (!absmax_scales) return BNB4_ERR_NULL;
+    if (!aligned16(absmax_scales)) return BNB4_ERR_ALIGN;
+    // absmax_q stands in the fp32 absmax's place for the common checks
+    bnb4_status s = check_matmul(x, W, reinterpret_cast<const float *>(absmax_q), bias, y, 1, N, K,
+                                 blocksize, qt, dt);
+    if (s != BNB4_OK) return s;
+    if (group < 32 || group > 4096 || (group & (group - 1)) != 0) return BNB4_ERR_BLOCKSIZE;
+    if (N > gemv_max_rows() || K > gemv_max_k()) return BNB4_ERR_SHAPE;
+    return from_cuda(launch_gemv(x, W, nullptr, absmax_q, absmax_scales, group, bias, y, N, K, blocksize,
+                                 qt, dt, stream));
 }
 
 bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, const void *bias,
@@ -134,6 +151,26 @@ bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *ab
     if (s != BNB4_OK) return s;
     if (N % 8 != 0) return BNB4_ERR_SHAPE;  // dY rows are TMA-loaded: 16-byte row pitch
     return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true, stream));
+}
+
+bnb4_status bnb4_double_quant(const float *absmax, int64_t n, int group, uint8_t *absmax_q,
+                              float *scales, cudaStream_t stream) {
+    if (n < 0) return BNB4_ERR_SHAPE;
+    if (group < 32 || group > 4096 || (group & (group - 1)) != 0) return BNB4_ERR_BLOCKSIZE;
+    if (n == 0) return BNB4_OK;
+    if (!absmax || !absmax_q || !scales) return BNB4_ERR_NULL;
+    if (!aligned16(absmax) || !aligned16(absmax_q) || !aligned16(scales)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_double_quant(absmax, n, group, absmax_q, scales, stream));
+}
+
+bnb4_status bnb4_dequant_absmax(const uint8_t *absmax_q, const float *scales, int64_t n, int group,
+                                float *absmax, cudaStream_t stream) {
+    if (n < 0) return BNB4_ERR_SHAPE;
+    if (group < 32 || group > 4096 || (group & (group - 1)) != 0) return BNB4_ERR_BLOCKSIZE;
+    if (n == 0) return BNB4_OK;
+    if (!absmax_q || !scales || !absmax) return BNB4_ERR_NULL;
+    if (!aligned16(absmax_q) || !aligned16(scales) || !aligned16(absmax)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_dequant_absmax(absmax_q, scales, n, group, absmax, stream));
 }
 
 bnb4_status bnb4_device_status(cudaStream_t stream) {

@@ -28,6 +28,15 @@
 //     xor-shuffles and added to the CTA's row sums in shared memory.
 // The codes enter as 16-bit values (the code table rounded once to bf16 /
 // fp16), as in the small-M kernel.  No global scratch.
+//
+// Double-quantized absmax ("mps-bitsandbytes 0.4.7", Functional API, Double
+// Quantization): with DQ the absmax array arrives as 8-bit codes plus one fp32
+// scale per group of consecutive blocks.  Each lane copies the aligned 32-bit
+// word holding its block's code (the slot keeps the same 16 B per lane) and
+// rebuilds absmax = RN(float(code) * RN(scale / 255)), the value the inverse
+// of the double quantization gives, so the product is the plain gemv's with
+// that absmax.  The weight stream shrinks from 4.5 to about 4.13 bits per
+// weight at blocks of 64.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,6 +52,7 @@ constexpr int kSlot = 4 * 32 * 16 + 32 * 16;  // W [4 rows][32 lanes] 16 B + abs
 constexpr int kLut = 256 * 32 * 4;            // 32 KB
 constexpr int kMaxRows = 1024;   // rows per CTA
 constexpr int kMaxK = 32768;
+constexpr int kXv = kMaxK / 8 / kThreads;     // 16-byte pieces of x per thread
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
@@ -55,6 +65,11 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     uint32_t v;
     asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
     return v;
+}
+
+// 4-byte copy of the first `n` bytes (0..4) at src, zero-filling the rest
+__device__ __forceinline__ void cp_async4_n(uint32_t dst, const void *src, int n) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(n));
 }
 
 template <int BYTES>
@@ -100,11 +115,14 @@ __device__ __forceinline__ int xswz(int k) {
     return (L << 5) | ((i ^ ((L >> 1) & 3)) << 3) | (k & 7);
 }
 
-template <typename D>
+// absmax: fp32 [N, K/B], or with DQ the 8-bit codes [N, K/B] (nq = N*K/B
+// bytes) with `scales` [ceil(nq / 2^log2G)]
+template <typename D, bool DQ>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
-            const float *__restrict__ absmax, const uint16_t *__restrict__ bias,
-            uint16_t *__restrict__ y, int N, int K, int log2B, const __grid_constant__ CodeTable tab) {
+            const void *__restrict__ absmax, const float *__restrict__ scales, int log2G,
+            const uint16_t *__restrict__ bias, uint16_t *__restrict__ y, int N, int K, int log2B,
+            const __grid_constant__ CodeTable tab) {
     extern __shared__ __align__(16) uint8_t smem[];
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
     uint8_t *ring = smem + kLut;                                                  // warps x STAGES
@@ -121,14 +139,6 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
     const int U = Q * S;
     const int64_t row_bytes = K >> 1;
     const int nblk = K >> log2B;
-
-    for (int e = tid >> 3; e < 256; e += kThreads / 8) {
-        const uint32_t v = Dt<D>::pack2(tab.v[e >> 4], tab.v[e & 15]);
-        reinterpret_cast<uint4 *>(lut + e * 32)[tid & 7] = make_uint4(v, v, v, v);
-    }
-    for (int k = tid; k < K; k += kThreads) xs[xswz(k)] = x[k];
-    for (int r = tid; r < rows; r += kThreads) rowsum[r] = 0.f;
-    __syncthreads();
 
     const uint32_t lut_base = (uint32_t)__cvta_generic_to_shared(lut);
     const uint32_t lane4 = 4u * lane;
@@ -148,16 +158,47 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             const bool v = ok && row < r1;
             cp_async<16>(base + (r * 32 + lane) * 16,
                          v ? W + (int64_t)row * row_bytes + (k >> 1) : W, v);
-            cp_async<4>(base + 4 * 32 * 16 + lane * 16 + 4 * r,
-                        v ? absmax + (int64_t)row * nblk + (k >> log2B) : absmax, v);
+            const int64_t bi = (int64_t)row * nblk + (k >> log2B);
+            if constexpr (DQ) {
+                const int64_t ws = bi & ~int64_t(3), left = (int64_t)N * nblk - ws;
+                cp_async4_n(base + 4 * 32 * 16 + lane * 16 + 4 * r,
+                            static_cast<const uint8_t *>(absmax) + (v ? ws : 0),
+                            v ? (left < 4 ? (int)left : 4) : 0);
+            } else {
+                cp_async<4>(base + 4 * 32 * 16 + lane * 16 + 4 * r,
+                            static_cast<const float *>(absmax) + (v ? bi : 0), v);
+            }
         }
     };
 
+    // the first weight copies go out before the table and x are staged, so
+    // their latency overlaps the prologue (the ring is per warp, nothing else
+    // touches it)
 #pragma unroll
     for (int i = 0; i < STAGES - 1; ++i) {
         issue(u_lo + i, i);
         cp_async_commit();
     }
+    {
+        // x: all 16-byte loads issued before any store (K <= kMaxK, K % 8 == 0)
+        const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
+        const int K8 = K >> 3;
+        uint4 xv[kXv];
+#pragma unroll
+        for (int i = 0; i < kXv; ++i)
+            if (tid + i * kThreads < K8) xv[i] = __ldg(x4 + tid + i * kThreads);
+        for (int e = tid >> 3; e < 256; e += kThreads / 8) {
+            const uint32_t v = Dt<D>::pack2(tab.v[e >> 4], tab.v[e & 15]);
+            reinterpret_cast<uint4 *>(lut + e * 32)[tid & 7] = make_uint4(v, v, v, v);
+        }
+        for (int r = tid; r < rows; r += kThreads) rowsum[r] = 0.f;
+#pragma unroll
+        for (int i = 0; i < kXv; ++i) {
+            const int c = tid + i * kThreads;
+            if (c < K8) *reinterpret_cast<uint4 *>(xs + xswz(8 * c)) = xv[i];
+        }
+    }
+    __syncthreads();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int q_cur = U > 0 ? u_lo / S : 0;
     for (int u = u_lo; u < u_hi; ++u) {
@@ -182,8 +223,19 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             for (int i = 0; i < 16; ++i) xq[i] = 0u;
         }
         const uint4 av = lds128(base + 4 * 32 * 16 + lane * 16);
-        const float am[4] = {__uint_as_float(av.x), __uint_as_float(av.y), __uint_as_float(av.z),
-                             __uint_as_float(av.w)};
+        float am[4] = {__uint_as_float(av.x), __uint_as_float(av.y), __uint_as_float(av.z),
+                       __uint_as_float(av.w)};
+        if constexpr (DQ) {
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int row = r0 + 4 * q + r;
+                const int64_t bi = (int64_t)row * nblk + (k >> log2B);
+                const float sc = (row < r1 && k < K) ? __ldg(scales + (bi >> log2G)) : 0.f;
+                const uint32_t code = (aw[r] >> (8 * (uint32_t)(bi & 3))) & 255u;
+                am[r] = __fmul_rn((float)code, __fdiv_rn(sc, 255.0f));
+            }
+        }
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const uint4 wv = lds128(base + (r * 32 + lane) * 16);
@@ -222,21 +274,22 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
     }
 }
 
-template <typename D>
-cudaError_t launch_t(const void *x, const uint8_t *W, const float *absmax, const void *bias,
-                     void *y, int N, int K, int log2B, const CodeTable &tab, cudaStream_t stream) {
+template <typename D, bool DQ>
+cudaError_t launch_t(const void *x, const uint8_t *W, const void *absmax, const float *scales, int log2G,
+                     const void *bias, void *y, int N, int K, int log2B, const CodeTable &tab,
+                     cudaStream_t stream) {
     const int G = device_sm_count();
     const int kpad = ((K + 31) / 32) * 32;
     const size_t smem = kLut + (size_t)kWarps * STAGES * kSlot + kMaxRows * 4 + (size_t)kpad * 2;
     static int smem_set = 0;  // largest dynamic shared memory size set so far
     if ((int)smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<D>,
+        cudaError_t e = cudaFuncSetAttribute(gemv_kernel<D, DQ>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         smem_set = (int)smem;
     }
-    gemv_kernel<D><<<G, kThreads, smem, stream>>>(
-        static_cast<const uint16_t *>(x), W, absmax, static_cast<const uint16_t *>(bias),
+    gemv_kernel<D, DQ><<<G, kThreads, smem, stream>>>(
+        static_cast<const uint16_t *>(x), W, absmax, scales, log2G, static_cast<const uint16_t *>(bias),
         static_cast<uint16_t *>(y), N, K, log2B, tab);
     return cudaGetLastError();
 }
@@ -246,16 +299,25 @@ cudaError_t launch_t(const void *x, const uint8_t *W, const float *absmax, const
 int64_t gemv_max_rows() { return (int64_t)device_sm_count() * kMaxRows; }
 int64_t gemv_max_k() { return kMaxK; }
 
-cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
-                        void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
-                        bnb4_dtype dt, cudaStream_t stream) {
+cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const uint8_t *absmax_q,
+                        const float *scales, int group, const void *bias, void *y, int64_t N,
+                        int64_t K, int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+                        cudaStream_t stream) {
     static const CodeTable nf4 = host_code_table(BNB4_NF4);
     static const CodeTable fp4 = host_code_table(BNB4_FP4);
     const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
     const int log2B = ilog2(blocksize);
+    if (absmax_q) {
+        const int log2G = ilog2(group);
+        if (dt == BNB4_F16)
+            return launch_t<F16, true>(x, W, absmax_q, scales, log2G, bias, y, (int)N, (int)K, log2B, tab,
+                                       stream);
+        return launch_t<BF16, true>(x, W, absmax_q, scales, log2G, bias, y, (int)N, (int)K, log2B, tab,
+                                    stream);
+    }
     if (dt == BNB4_F16)
-        return launch_t<F16>(x, W, absmax, bias, y, (int)N, (int)K, log2B, tab, stream);
-    return launch_t<BF16>(x, W, absmax, bias, y, (int)N, (int)K, log2B, tab, stream);
+        return launch_t<F16, false>(x, W, absmax, nullptr, 0, bias, y, (int)N, (int)K, log2B, tab, stream);
+    return launch_t<BF16, false>(x, W, absmax, nullptr, 0, bias, y, (int)N, (int)K, log2B, tab, stream);
 }
 
 }  // namespace bnb4

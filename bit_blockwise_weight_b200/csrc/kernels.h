@@ -23,11 +23,15 @@ cudaError_t launch_dequantize(const uint8_t *packed, const float *absmax, void *
 // M == 1, CUDA cores; handles N <= gemv_max_rows() and K <= gemv_max_k()
 int64_t gemv_max_rows();
 int64_t gemv_max_k();
-cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
-                        void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
-                        bnb4_dtype dt, cudaStream_t stream);
+// absmax_q == nullptr: fp32 absmax; else 8-bit double-quantized absmax codes
+// with one fp32 scale per `group` codes (absmax unused)
+cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, const uint8_t *absmax_q,
+                        const float *scales, int group, const void *bias, void *y, int64_t N,
+                        int64_t K, int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+                        cudaStream_t stream);
 
-// 1 <= M <= 16: weights decoded into tensor memory, tcgen05.mma with N = 16 tokens
+// 1 <= M <= 16: TMA-staged weights decoded in registers, mma.sync with the
+// 16-row token tile
 cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
                               const void *bias, void *Y, int64_t M, int64_t N, int64_t K,
                               int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
@@ -39,6 +43,13 @@ cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax,
                            const void *bias, void *D, int64_t M, int64_t N, int64_t K,
                            int blocksize, bnb4_quant_type qt, bnb4_dtype dt, bool backward,
                            cudaStream_t stream);
+
+// double quantization of an absmax array (groups of `group`, a power of two
+// in [32, 4096]) and its inverse
+cudaError_t launch_double_quant(const float *absmax, int64_t n, int group, uint8_t *q, float *scales,
+                                cudaStream_t stream);
+cudaError_t launch_dequant_absmax(const uint8_t *q, const float *scales, int64_t n, int group, float *out,
+                                  cudaStream_t stream);
 
 // read and clear the count of bounded waits that gave up, per kernel file
 cudaError_t gemm_tc_take_timeouts(unsigned int *count);

@@ -61,6 +61,18 @@ def roundtrip_tensor(n: int, seed: int, dtype: str, device: str = "cpu") -> torc
     return normal((n,), seed, 1.0, dtype, outlier_frac=0.01, outlier_scale=20.0, device=device)
 
 
+def absmax_values(n: int, seed: int = 4, sigma: float = 0.02, zero_frac: float = 0.0) -> torch.Tensor:
+    """n positive fp32 values shaped like the block maxima of N(0, sigma) weights
+    (about 2.4 sigma for blocks of 64, a narrow spread): sigma * 2.4 *
+    exp(0.15 * randn).  With zero_frac > 0, a ``torch.rand(n) < zero_frac``
+    mask drawn after that sets values to 0 (all-zero blocks)."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    a = torch.exp(torch.randn(n, generator=g, dtype=torch.float32) * 0.15) * (2.4 * sigma)
+    if zero_frac > 0.0:
+        a[torch.rand(n, generator=g) < zero_frac] = 0.0
+    return a
+
+
 def storage_numpy(t: torch.Tensor):
     """Raw storage as numpy: float32 stays float32, 16-bit types become uint16 bits."""
     t = t.contiguous().cpu()

@@ -18,6 +18,11 @@
  *   bnb4_gemm_backward  "Feat/mps gemm 4bit bf16", What runs natively now and
  *                       the paragraph on the new op: grad_input =
  *                       grad_output @ dequantize_4bit(B).
+ *   bnb4_double_quant,  "mps-bitsandbytes 0.4.7", Functional API, Double
+ *   bnb4_dequant_absmax Quantization (double_quant(absmax,
+ *                       double_quant_block=256), dequant_absmax).
+ *   bnb4_gemv_dq        gemv_4bit whose weight carries the double-quantized
+ *                       absmax of the same section (8-bit statistics).
  *
  * Numeric contract (the readings of the pages that the CPU oracle follows):
  *   - absmax[b] = max |x_i| over block b, in fp32; blocks are `blocksize`
@@ -130,6 +135,24 @@ bnb4_status bnb4_gemv(const void *x, const uint8_t *packedW,
                       cudaStream_t stream);
 
 /*
+ * bnb4_gemv with a double-quantized absmax (see bnb4_double_quant): the
+ * weight's absmax array [N, K/blocksize], flattened, arrives as its 8-bit
+ * codes absmax_q [N*K/blocksize] and absmax_scales [ceil(N*K/blocksize /
+ * group)].  The result equals bnb4_gemv's with absmax =
+ * bnb4_dequant_absmax(absmax_q, absmax_scales) (the kernel rebuilds each
+ * block's absmax with the same two fp32 operations), reading 1 + 4/group
+ * bytes of absmax per block instead of 4.
+ *   Same constraints as bnb4_gemv, plus group in {32, ..., 4096} (a power of
+ *   two; 256 is the pages' default) and N <= 148 * 1024 (one row slab per
+ *   SM), K <= 32768 (BNB4_ERR_SHAPE otherwise).
+ */
+bnb4_status bnb4_gemv_dq(const void *x, const uint8_t *packedW,
+                         const uint8_t *absmax_q, const float *absmax_scales,
+                         int group, const void *bias, void *y, int64_t N,
+                         int64_t K, int blocksize, bnb4_quant_type quant_type,
+                         bnb4_dtype dt, cudaStream_t stream);
+
+/*
  * General matmul: Y[M, N] = X[M, K] @ dequant(W)^T (+ bias), row-major.
  *   X [M, K] of dt;  bias [N] of dt or NULL;  Y [M, N] of dt (out).
  *   Same constraints as bnb4_gemv; M >= 1.  Small M streams the weight once
@@ -154,6 +177,32 @@ bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *packedW,
                                int64_t N, int64_t K, int blocksize,
                                bnb4_quant_type quant_type, bnb4_dtype dt,
                                cudaStream_t stream);
+
+/*
+ * Double quantization of an absmax array (the pages give the call and the
+ * group of 256, not the arithmetic; this is the plainest reading).  For each
+ * group of `group` consecutive values (the last one may be short):
+ *   scales[g] = the group maximum in fp32 (values not above the running
+ *               maximum, NaN included, are skipped; +0 if none is > 0);
+ *   absmax_q[i] = clamp(rint(RN(RN(absmax[i] / scales[g]) * 255)), 0, 255),
+ *               rint ties to even, NaN -> 0, and 0 when scales[g] == 0.
+ *   absmax   [n] float32, absmax_q [n] uint8 (out), scales [ceil(n/group)]
+ *            float32 (out); all 16-byte aligned.
+ *   group in {32, 64, ..., 4096} (256 is the pages' default); n >= 0.
+ * 8 + 32/group bits per scale instead of 32.
+ */
+bnb4_status bnb4_double_quant(const float *absmax, int64_t n, int group,
+                              uint8_t *absmax_q, float *scales,
+                              cudaStream_t stream);
+
+/*
+ * Inverse of bnb4_double_quant:
+ *   absmax[i] = RN(float(absmax_q[i]) * RN(scales[i / group] / 255)).
+ * Same arguments and constraints (absmax is the [n] float32 output).
+ */
+bnb4_status bnb4_dequant_absmax(const uint8_t *absmax_q, const float *scales,
+                                int64_t n, int group, float *absmax,
+                                cudaStream_t stream);
 
 /*
  * Device-side status of the library's kernels (no counterpart on the pages:

@@ -10,7 +10,8 @@
 //           NaN -> 0, and 0 when scale == 0;
 //   inverse: out = RN(float(q) * RN(scale / 255)).
 // An unsigned linear 8-bit code (absmax values are >= 0); every step is one
-// IEEE fp32 operation, so the results are bit-exact.
+// correctly rounded fp32 operation (RN(scale / 255) by div255_rn), so the
+// results are bit-exact.
 //
 // Both kernels are HBM-bound streams.  double_quant: one warp per group, its
 // lanes reading and writing consecutive elements (coalesced), the maximum by
@@ -72,13 +73,13 @@ dequant_absmax_kernel(const uint8_t *__restrict__ q, const float *__restrict__ s
         if (i0 + 4 <= n) {
             const uchar4 c = __ldcs(reinterpret_cast<const uchar4 *>(q + i0));
             // four consecutive values never straddle a group (G >= 32)
-            const float step = __fdiv_rn(scales[i0 >> log2G], 255.0f);
+            const float step = div255_rn(scales[i0 >> log2G]);
             __stcs(reinterpret_cast<float4 *>(out + i0),
                    make_float4(__fmul_rn((float)c.x, step), __fmul_rn((float)c.y, step),
                                __fmul_rn((float)c.z, step), __fmul_rn((float)c.w, step)));
         } else {
             for (int64_t i = i0; i < n; ++i)
-                out[i] = __fmul_rn((float)q[i], __fdiv_rn(scales[i >> log2G], 255.0f));
+                out[i] = __fmul_rn((float)q[i], div255_rn(scales[i >> log2G]));
         }
     }
 }

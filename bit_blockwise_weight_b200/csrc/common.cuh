@@ -171,4 +171,22 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
 
+// RN(s / 255) in fp32 (the step of a double-quantized absmax) without a
+// divide: Markstein's correction (P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", 1990): with y = RN(1/255)
+// and q0 = RN(s y), the residual s - 255 q0 is exact in one fma and
+// RN(q0 + residual * y) is the correctly rounded quotient.  Used for s == 0
+// and 2^-100 <= s <= 2^100, where no step underflows (checked against IEEE
+// division over every fp32 significand); other values (negative, tiny,
+// huge, inf, NaN) take the IEEE divide.
+__device__ __forceinline__ float div255_rn(float s) {
+    if (s == 0.0f || (s >= 0x1p-100f && s <= 0x1p100f)) {
+        const float y = 0x1.010102p-8f;  // RN(1/255)
+        const float q0 = __fmul_rn(s, y);
+        const float r = __fmaf_rn(-q0, 255.0f, s);
+        return __fmaf_rn(r, y, q0);
+    }
+    return __fdiv_rn(s, 255.0f);
+}
+
 }  // namespace bnb4

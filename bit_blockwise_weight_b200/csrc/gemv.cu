@@ -25,18 +25,22 @@
 //   * the lane's 32 weights lie in one quantization block: their sum is
 //     scaled by the block absmax once, in fp32;
 //   * when a warp leaves a quad, its 4 row sums are reduced across lanes with
-//     xor-shuffles and added to the CTA's row sums in shared memory.
+//     xor-shuffles and stored to shared memory; quads shared by neighbouring
+//     warps are added in warp order at the end (the result is the same bits
+//     on every run).
 // The codes enter as 16-bit values (the code table rounded once to bf16 /
 // fp16), as in the small-M kernel.  No global scratch.
 //
 // Double-quantized absmax ("mps-bitsandbytes 0.4.7", Functional API, Double
 // Quantization): with DQ the absmax array arrives as 8-bit codes plus one fp32
-// scale per group of consecutive blocks.  Each lane copies the aligned 32-bit
-// word holding its block's code (the slot keeps the same 16 B per lane) and
-// rebuilds absmax = RN(float(code) * RN(scale / 255)), the value the inverse
-// of the double quantization gives, so the product is the plain gemv's with
-// that absmax.  The weight stream shrinks from 4.5 to about 4.13 bits per
-// weight at blocks of 64.
+// scale per group of consecutive blocks.  Lanes 2i and 2i+1 share a block
+// (blocks hold 64 or more weights); for the unit's 4 rows the even lane copies
+// the aligned 32-bit words holding the block's codes and the odd lane the
+// scales, into their two 16-byte slot entries (the slot keeps its size).  Both
+// lanes rebuild absmax = RN(float(code) * RN(scale / 255)), the value the
+// inverse of the double quantization gives, so the product is the plain
+// gemv's with that absmax.  The weight stream shrinks from 4.5 to about 4.13
+// bits per weight at blocks of 64.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -127,7 +131,8 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
     uint32_t *lut = reinterpret_cast<uint32_t *>(smem);
     uint8_t *ring = smem + kLut;                                                  // warps x STAGES
     float *rowsum = reinterpret_cast<float *>(ring + kWarps * STAGES * kSlot);    // [kMaxRows]
-    uint16_t *xs = reinterpret_cast<uint16_t *>(rowsum + kMaxRows);              // [K] swizzled
+    float *part = rowsum + kMaxRows;                                              // [kWarps][2][4]
+    uint16_t *xs = reinterpret_cast<uint16_t *>(part + kWarps * 8);              // [K] swizzled
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x;
@@ -158,13 +163,19 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             const bool v = ok && row < r1;
             cp_async<16>(base + (r * 32 + lane) * 16,
                          v ? W + (int64_t)row * row_bytes + (k >> 1) : W, v);
-            const int64_t bi = (int64_t)row * nblk + (k >> log2B);
             if constexpr (DQ) {
-                const int64_t ws = bi & ~int64_t(3), left = (int64_t)N * nblk - ws;
-                cp_async4_n(base + 4 * 32 * 16 + lane * 16 + 4 * r,
-                            static_cast<const uint8_t *>(absmax) + (v ? ws : 0),
-                            v ? (left < 4 ? (int)left : 4) : 0);
+                // even lane: the word holding the block's code; odd lane: the
+                // block's group scale (one copy either way, no divergence).
+                // Block indices fit in 32 bits: N * K / B <= 151552 * 512.
+                const int bi = row * nblk + (k >> log2B);
+                const int ws = bi & ~3, left = N * nblk - ws;
+                const void *src = (lane & 1) ? static_cast<const void *>(scales + (v ? bi >> log2G : 0))
+                                             : static_cast<const void *>(static_cast<const uint8_t *>(absmax) +
+                                                                         (v ? ws : 0));
+                cp_async4_n(base + 4 * 32 * 16 + lane * 16 + 4 * r, src,
+                            !v ? 0 : (lane & 1) ? 4 : (left < 4 ? left : 4));
             } else {
+                const int64_t bi = (int64_t)row * nblk + (k >> log2B);
                 cp_async<4>(base + 4 * 32 * 16 + lane * 16 + 4 * r,
                             static_cast<const float *>(absmax) + (v ? bi : 0), v);
             }
@@ -191,7 +202,6 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             const uint32_t v = Dt<D>::pack2(tab.v[e >> 4], tab.v[e & 15]);
             reinterpret_cast<uint4 *>(lut + e * 32)[tid & 7] = make_uint4(v, v, v, v);
         }
-        for (int r = tid; r < rows; r += kThreads) rowsum[r] = 0.f;
 #pragma unroll
         for (int i = 0; i < kXv; ++i) {
             const int c = tid + i * kThreads;
@@ -200,7 +210,6 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
     }
     __syncthreads();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    int q_cur = U > 0 ? u_lo / S : 0;
     for (int u = u_lo; u < u_hi; ++u) {
         const int it = u - u_lo;
         issue(u + STAGES - 1, (it + STAGES - 1) % STAGES);
@@ -226,14 +235,19 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
         float am[4] = {__uint_as_float(av.x), __uint_as_float(av.y), __uint_as_float(av.z),
                        __uint_as_float(av.w)};
         if constexpr (DQ) {
-            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+            // the lane pair's code words and scales (zeros for rows past the slab
+            // or segments past K, whose sums are dropped or zero)
+            const uint32_t pb = base + 4 * 32 * 16 + (lane & ~1) * 16;
+            const uint4 cw = lds128(pb), sw = lds128(pb + 16);
+            const uint32_t aw[4] = {cw.x, cw.y, cw.z, cw.w};
+            const uint32_t sc[4] = {sw.x, sw.y, sw.z, sw.w};
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const int row = r0 + 4 * q + r;
-                const int64_t bi = (int64_t)row * nblk + (k >> log2B);
-                const float sc = (row < r1 && k < K) ? __ldg(scales + (bi >> log2G)) : 0.f;
-                const uint32_t code = (aw[r] >> (8 * (uint32_t)(bi & 3))) & 255u;
-                am[r] = __fmul_rn((float)code, __fdiv_rn(sc, 255.0f));
+                const int bi = (r0 + 4 * q + r) * nblk + (k >> log2B);
+                // byte (bi & 3) of the word into the low byte of 0x4b000000:
+                // the float 2^23 + code, exact
+                const float c = __uint_as_float(__byte_perm(aw[r], 0x4b000000u, 0x7440u | (bi & 3)));
+                am[r] = __fmul_rn(__fsub_rn(c, 8388608.0f), div255_rn(__uint_as_float(sc[r])));
             }
         }
 #pragma unroll
@@ -253,22 +267,38 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
             }
             acc[r] = __fmaf_rn(s0 + s1, am[r], acc[r]);
         }
-        // leaving this quad: fold the lane sums into the CTA's row sums
+        // leaving this quad: reduce the lane sums.  A quad strictly inside the
+        // warp's range is the warp's alone and goes straight to the row sums;
+        // the first and last quads may be shared with neighbouring warps and
+        // go to this warp's two partial slots, added below in warp order, so
+        // that the result does not depend on which warp finishes first.
         if (u + 1 == u_hi || (u + 1) / S != q) {
+            const int qf = u_lo / S, ql = (u_hi - 1) / S;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const float v = warp_sum(acc[r]);
                 const int row = 4 * q + r;
-                if (lane == 0 && row < rows) atomicAdd(&rowsum[row], v);
+                if (lane == 0) {
+                    if (q == qf) part[warp * 8 + r] = v;
+                    else if (q == ql) part[warp * 8 + 4 + r] = v;
+                    else if (row < rows) rowsum[row] = v;
+                }
                 acc[r] = 0.f;
             }
         }
-        (void)q_cur;
     }
     cp_async_wait<0>();
     __syncthreads();
     for (int r = tid; r < rows; r += kThreads) {
-        float v = rowsum[r];
+        // the warps whose unit ranges meet this row's quad, in order
+        const int q = r >> 2, ul = q * S, uh = ul + S;
+        float v = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+            const int lo = (int)(((int64_t)U * w) / kWarps), hi = (int)(((int64_t)U * (w + 1)) / kWarps);
+            if (lo >= hi || hi <= ul || lo >= uh) continue;
+            const int qf = lo / S, ql = (hi - 1) / S;
+            v += q == qf ? part[w * 8 + (r & 3)] : q == ql ? part[w * 8 + 4 + (r & 3)] : rowsum[r];
+        }
         if (bias) v += Dt<D>::to_f32(bias[r0 + r]);
         y[r0 + r] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);
     }
@@ -280,7 +310,7 @@ cudaError_t launch_t(const void *x, const uint8_t *W, const void *absmax, const 
                      cudaStream_t stream) {
     const int G = device_sm_count();
     const int kpad = ((K + 31) / 32) * 32;
-    const size_t smem = kLut + (size_t)kWarps * STAGES * kSlot + kMaxRows * 4 + (size_t)kpad * 2;
+    const size_t smem = kLut + (size_t)kWarps * STAGES * kSlot + kMaxRows * 4 + kWarps * 8 * 4 + (size_t)kpad * 2;
     static int smem_set = 0;  // largest dynamic shared memory size set so far
     if ((int)smem > smem_set) {
         cudaError_t e = cudaFuncSetAttribute(gemv_kernel<D, DQ>,

@@ -158,3 +158,28 @@ def test_gemv_dq_argument_checks():
     assert bnb4.bnb4_gemv_dq(*args(g=48)) == 3
     assert bnb4.bnb4_gemv_dq(*args(K=40 * 1024)) == 4
     torch.cuda.synchronize()
+
+
+def test_dequant_absmax_every_significand():
+    """The inverse's step RN(scale / 255) for every fp32 significand (scales in
+    [1, 2)), and random significands at the exponents around the kernel's
+    fast-division range (2^-101 .. 2^101) and in the subnormals: code 1 gives
+    the step itself, codes 255 and 128 its products."""
+    G = 32
+    rng = np.random.default_rng(7)
+    edge = []
+    for e in (-126, -102, -101, -100, -99, -60, 60, 99, 100, 101, 126):
+        m = rng.integers(0, 1 << 23, 4096, dtype=np.uint32)
+        edge.append(((np.uint32(e + 127) << 23) | m).view(np.float32))
+    edge.append(rng.integers(1, 1 << 23, 4096, dtype=np.uint32).view(np.float32))  # subnormals
+    edge.append(np.array([0.0, np.inf, np.float32(2.0 ** -100), np.float32(2.0 ** 100)], np.float32))
+    chunks = [((np.uint32(127) << 23) | np.arange(c << 21, (c + 1) << 21, dtype=np.uint32)).view(np.float32)
+              for c in range(4)] + [np.concatenate(edge)]
+    for sc in chunks:
+        n = sc.size * G
+        q = np.zeros(n, np.uint8)
+        q[0::G], q[1::G], q[2::G] = 1, 255, 128
+        got = to_host(bnb4.dequant_absmax(torch.from_numpy(q).cuda(), torch.from_numpy(sc).cuda(), G))
+        want = oracle.dequant_absmax(q, sc, G)
+        for o in range(3):
+            assert _same_bits(got[o::G], want[o::G]), o

@@ -210,6 +210,7 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
     }
     __syncthreads();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int qf = U > 0 ? u_lo / S : 0, ql = U > 0 ? (u_hi - 1) / S : 0;  // this warp's first and last quads
     for (int u = u_lo; u < u_hi; ++u) {
         const int it = u - u_lo;
         issue(u + STAGES - 1, (it + STAGES - 1) % STAGES);
@@ -273,7 +274,6 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
         // go to this warp's two partial slots, added below in warp order, so
         // that the result does not depend on which warp finishes first.
         if (u + 1 == u_hi || (u + 1) / S != q) {
-            const int qf = u_lo / S, ql = (u_hi - 1) / S;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 const float v = warp_sum(acc[r]);
@@ -290,14 +290,18 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W,
     cp_async_wait<0>();
     __syncthreads();
     for (int r = tid; r < rows; r += kThreads) {
-        // the warps whose unit ranges meet this row's quad, in order
+        // the warps whose unit ranges meet this row's quad (units [ul, uh)), in
+        // order: from the warp holding unit ul to the one holding uh - 1 (unit u
+        // lies in warp ceil(kWarps (u + 1) / U) - 1).  A warp starting inside the
+        // quad left it in slot 0, one ending inside it in slot 1; otherwise the
+        // quad is the warp's alone.
         const int q = r >> 2, ul = q * S, uh = ul + S;
+        const int w0 = (kWarps * (ul + 1) + U - 1) / U - 1, w1 = (kWarps * uh + U - 1) / U - 1;
         float v = 0.f;
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = w0; w <= w1; ++w) {
             const int lo = (int)(((int64_t)U * w) / kWarps), hi = (int)(((int64_t)U * (w + 1)) / kWarps);
-            if (lo >= hi || hi <= ul || lo >= uh) continue;
-            const int qf = lo / S, ql = (hi - 1) / S;
-            v += q == qf ? part[w * 8 + (r & 3)] : q == ql ? part[w * 8 + 4 + (r & 3)] : rowsum[r];
+            if (lo >= hi) continue;
+            v += lo >= ul ? part[w * 8 + (r & 3)] : hi - 1 < uh ? part[w * 8 + 4 + (r & 3)] : rowsum[r];
         }
         if (bias) v += Dt<D>::to_f32(bias[r0 + r]);
         y[r0 + r] = (uint16_t)(Dt<D>::pack2(v, 0.f) & 0xffffu);

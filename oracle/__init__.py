@@ -61,6 +61,9 @@ def lib() -> ctypes.CDLL:
             "oracle_matmul_backward_entries": (I, [P, I, P, P, I64, I64, I64, I, I, P, P, I64, P]),
             "oracle_double_quant": (I, [P, I64, I, P, P]),
             "oracle_dequant_absmax": (I, [P, P, I64, I, P]),
+            "oracle_quantize_8bit": (I, [P, I, I64, I, P, P, P]),
+            "oracle_dequantize_8bit": (I, [P, P, I64, I, P, I, P]),
+            "oracle_embedding_4bit": (I, [P, P, I64, I64, I, I, P, I64, I, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -212,3 +215,50 @@ def dequant_absmax(q, scales, group=256):
     _check(lib().oracle_dequant_absmax(_ptr(q), _ptr(scales), q.size, group, _ptr(out)),
            "dequant_absmax")
     return out
+
+
+def _code8(code) -> np.ndarray:
+    code = np.ascontiguousarray(code, np.float32).reshape(-1)
+    if code.size != 256:
+        raise ValueError("an 8-bit code table has 256 entries")
+    return code
+
+
+def quantize_8bit(x: np.ndarray, dtype: str, blocksize: int, code) -> tuple:
+    """R10: (q uint8[n], absmax float32[ceil(n/blocksize)]) against a 256-entry table."""
+    x = _as_storage(x, dtype).reshape(-1)
+    code = _code8(code)
+    if blocksize <= 0:
+        raise ValueError("blocksize must be positive")
+    q = np.zeros(x.size, np.uint8)
+    absmax = np.zeros((x.size + blocksize - 1) // blocksize, np.float32)
+    _check(lib().oracle_quantize_8bit(_ptr(x), DTYPES[dtype], x.size, blocksize, _ptr(code),
+                                      _ptr(q), _ptr(absmax)), "quantize_8bit")
+    return q, absmax
+
+
+def dequantize_8bit(q: np.ndarray, absmax: np.ndarray, n: int, blocksize: int, code,
+                    out_dtype: str) -> np.ndarray:
+    """R10 inverse: out[i] = RN_out(fp32(code[q[i]] * absmax[i // blocksize]))."""
+    q = np.ascontiguousarray(q, np.uint8).reshape(-1)
+    absmax = np.ascontiguousarray(absmax, np.float32).reshape(-1)
+    code = _code8(code)
+    assert q.size >= n and absmax.size >= (n + blocksize - 1) // blocksize
+    out = np.empty(n, np.float32 if out_dtype == "f32" else np.uint16)
+    _check(lib().oracle_dequantize_8bit(_ptr(q), _ptr(absmax), n, blocksize, _ptr(code),
+                                        DTYPES[out_dtype], _ptr(out)), "dequantize_8bit")
+    return out
+
+
+def embedding_4bit(packed: np.ndarray, absmax: np.ndarray, V: int, D: int, blocksize: int,
+                   qtype: str, idx, out_dtype: str) -> np.ndarray:
+    """R11: rows idx of a [V, D] table quantized as one flat array -> [len(idx), D]."""
+    packed = np.ascontiguousarray(packed, np.uint8).reshape(-1)
+    absmax = np.ascontiguousarray(absmax, np.float32).reshape(-1)
+    idx = np.ascontiguousarray(idx, np.int64).reshape(-1)
+    assert packed.size >= (V * D + 1) // 2 and absmax.size >= (V * D + blocksize - 1) // blocksize
+    out = np.empty(idx.size * D, np.float32 if out_dtype == "f32" else np.uint16)
+    _check(lib().oracle_embedding_4bit(_ptr(packed), _ptr(absmax), V, D, blocksize, QTYPES[qtype],
+                                       _ptr(idx), idx.size, DTYPES[out_dtype], _ptr(out)),
+           "embedding_4bit")
+    return out.reshape(idx.size, D)

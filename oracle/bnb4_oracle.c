@@ -30,6 +30,11 @@
  *      round-to-nearest-even conversion to the output dtype.
  *   R8 matmul reference: float64 sum over k of x * fp32(code * absmax), plus
  *      bias, with no rounding of the result.
+ *   R9 double quantization of absmax (see oracle_double_quant).
+ *   R10 8-bit blockwise: steps R3-R5 and R7 with a caller's 256-entry code
+ *      table and one code index per byte (see oracle_quantize_8bit).
+ *   R11 4-bit embedding lookup: rows of a table quantized as one flat array
+ *      (see oracle_embedding_4bit).
  */
 #include "bnb4_oracle.h"
 
@@ -411,5 +416,108 @@ int oracle_dequant_absmax(const uint8_t *q, const float *scales, int64_t n,
         const float step = scales[i / group] / 255.0f;  /* fp32 quotient */
         out[i] = (float)q[i] * step;                    /* fp32 product */
     }
+    return 0;
+}
+
+/* ---------------------------------------- 8-bit blockwise quantization (R10) */
+
+/* A caller's table is usable when it is strictly ascending, finite, inside
+ * [-1, 1], and every entry is 0 or at least 2^-24 in magnitude.  With the
+ * last condition every comparison of |v - c| that can decide an index is
+ * exact in float64: a close call sits at a midpoint of two entries, which is
+ * then at least 2^-25 in magnitude, and the differences of fp32 values that
+ * large span fewer than 53 bits. */
+static int code8_usable(const float *code)
+{
+    for (int j = 0; j < 256; ++j) {
+        const float c = code[j];
+        if (!(c >= -1.0f && c <= 1.0f))
+            return 0;
+        if (c != 0.0f && fabsf(c) < 0x1p-24f)
+            return 0;
+        if (j > 0 && !(code[j - 1] < c))
+            return 0;
+    }
+    return 1;
+}
+
+/* R10 (as R5): exact nearest of the 256 entries, ties to the smallest index. */
+static int nearest_code8(float v, const float *code)
+{
+    int best_j = 0;
+    double best_d = fabs((double)v - (double)code[0]);
+    for (int j = 1; j < 256; ++j) {
+        const double dist = fabs((double)v - (double)code[j]);
+        if (dist < best_d) {
+            best_d = dist;
+            best_j = j;
+        }
+    }
+    return best_j;
+}
+
+int oracle_quantize_8bit(const void *x, int dtype, int64_t n, int blocksize,
+                         const float *code, uint8_t *q, float *absmax)
+{
+    if (!code8_usable(code) || !valid_dtype(dtype) || blocksize <= 0 || n < 0)
+        return -1;
+    const int64_t nblocks = (n + blocksize - 1) / blocksize;
+    for (int64_t b = 0; b < nblocks; ++b) {
+        const int64_t lo = b * blocksize;
+        const int64_t hi = lo + blocksize < n ? lo + blocksize : n; /* R3 tail */
+        /* step 1 (R3): block absmax */
+        float amax = 0.0f;
+        for (int64_t i = lo; i < hi; ++i) {
+            const float mag = fabsf(load_elem(x, dtype, i));
+            if (mag > amax)
+                amax = mag;
+        }
+        absmax[b] = amax;
+        for (int64_t i = lo; i < hi; ++i) {
+            /* step 2 (R4): normalise */
+            const float xi = load_elem(x, dtype, i);
+            const float v = (amax == 0.0f) ? 0.0f : xi / amax;
+            /* step 3 (R10): nearest entry, one byte per element */
+            q[i] = (uint8_t)nearest_code8(v, code);
+        }
+    }
+    return 0;
+}
+
+int oracle_dequantize_8bit(const uint8_t *q, const float *absmax, int64_t n,
+                           int blocksize, const float *code, int out_dtype,
+                           void *out)
+{
+    if (!code8_usable(code) || !valid_dtype(out_dtype) || blocksize <= 0 || n < 0)
+        return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        /* R7: one fp32 product, then the output rounding */
+        const float entry = code[q[i]];
+        const float scale = absmax[i / blocksize];
+        store_elem(out, out_dtype, i, entry * scale);
+    }
+    return 0;
+}
+
+/* ------------------------------------------ 4-bit embedding lookup (R11) */
+
+int oracle_embedding_4bit(const uint8_t *packed, const float *absmax, int64_t V,
+                          int64_t D, int blocksize, int qtype,
+                          const int64_t *idx, int64_t n_idx, int out_dtype,
+                          void *out)
+{
+    float code[16];
+    if (oracle_code_table(qtype, code) != 0 || !valid_dtype(out_dtype) ||
+        blocksize <= 0 || V < 0 || D < 0 || n_idx < 0)
+        return -1;
+    for (int64_t r = 0; r < n_idx; ++r) /* every index checked before any output */
+        if (idx[r] < 0 || idx[r] >= V)
+            return -1;
+    for (int64_t r = 0; r < n_idx; ++r)
+        for (int64_t k = 0; k < D; ++k) {
+            /* element k of table row idx[r] is element idx[r]*D + k of the flat array */
+            const int64_t e = idx[r] * D + k;
+            store_elem(out, out_dtype, r * D + k, dequant_f32(packed, absmax, e, blocksize, code));
+        }
     return 0;
 }

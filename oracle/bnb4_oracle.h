@@ -1,6 +1,8 @@
 /*
  * bnb4_oracle.h -- plain, slow CPU oracle for 4-bit blockwise weight
- * quantization (NF4 / FP4) and the matmuls that consume it.
+ * quantization (NF4 / FP4) and the matmuls that consume it, with the
+ * double-quantized absmax, 8-bit blockwise quantization and the 4-bit
+ * embedding lookup.
  *
  * TEST INFRASTRUCTURE ONLY.  This header and bnb4_oracle.c are used by the
  * test suite, by the smoke check and by the benchmark's CPU-baseline leg.
@@ -100,6 +102,37 @@ int oracle_double_quant(const float *absmax, int64_t n, int group, uint8_t *q,
                         float *scales);
 int oracle_dequant_absmax(const uint8_t *q, const float *scales, int64_t n,
                           int group, float *out);
+
+/* R10 -- 8-bit blockwise quantization ("Feat/mps gemm 4bit bf16", What
+ * runs natively now: quantize_blockwise / dequantize_blockwise; Correctness:
+ * the exact float64 reference, never a lookup table).  The pages print no
+ * 8-bit code table, so the table is the caller's: code[256] strictly
+ * ascending, finite, in [-1, 1], each entry 0 or at least 2^-24 in magnitude
+ * (otherwise -1).  Per block of `blocksize` elements (the last may be short):
+ * absmax as R3, v = x / absmax as R4, q[i] = argmin_j |v - code[j]| in
+ * float64 with ties to the smallest j (one byte per element).
+ *   x [n] of dtype; q [n] uint8 (out); absmax [ceil(n/blocksize)] (out).
+ * Return 0, or -1 on a bad argument. */
+int oracle_quantize_8bit(const void *x, int dtype, int64_t n, int blocksize,
+                         const float *code, uint8_t *q, float *absmax);
+
+/* R10 inverse: out[i] = RN_out_dtype(fp32(code[q[i]] * absmax[i/blocksize])). */
+int oracle_dequantize_8bit(const uint8_t *q, const float *absmax, int64_t n,
+                           int blocksize, const float *code, int out_dtype,
+                           void *out);
+
+/* R11 -- 4-bit embedding lookup ("mps-bitsandbytes 0.4.7", Quantized
+ * Embeddings: Embedding4bit.from_embedding quantizes an embedding table, NF4
+ * by default).  The [V, D] table was quantized as one flat array of V*D
+ * elements (R3-R6); row r of the output is table row idx[r] dequantized as
+ * R7: out[r*D + k] = dequantized element idx[r]*D + k.
+ *   packed [ceil(V*D/2)], absmax [ceil(V*D/blocksize)], idx [n_idx] int64,
+ *   out [n_idx * D] of out_dtype.
+ * Every index must lie in [0, V); otherwise -1 and out is untouched. */
+int oracle_embedding_4bit(const uint8_t *packed, const float *absmax, int64_t V,
+                          int64_t D, int blocksize, int qtype,
+                          const int64_t *idx, int64_t n_idx, int out_dtype,
+                          void *out);
 
 #ifdef __cplusplus
 }

@@ -127,3 +127,26 @@ def matmul(X: list, W: list, bias=None) -> list:
         Y.append([sum((a * b for a, b in zip(row, wr)), Fraction(0)) + (bias[j] if bias else 0)
                   for j, wr in enumerate(W)])
     return Y
+
+
+def quantize_with_table(values: list, blocksize: int, codes: list):
+    """Blockwise quantization against any ascending table of exact Fractions:
+    (code indices, absmax list), one index per element, ties to the smallest index."""
+    idxs, absmax = [], []
+    for lo in range(0, len(values), blocksize):
+        blk = values[lo:lo + blocksize]
+        a = max(abs(v) for v in blk)
+        absmax.append(a)
+        for x in blk:
+            v = Fraction(0) if a == 0 else round_to(x / a, "f32")
+            best = min(range(len(codes)), key=lambda i: (abs(v - codes[i]), i))
+            idxs.append(best)
+    return idxs, absmax
+
+
+def dequantize_with_table(idxs: list, absmax: list, blocksize: int, codes: list, out_fmt: str) -> list:
+    out = []
+    for i, q in enumerate(idxs):
+        p = round_to(codes[q] * absmax[i // blocksize], "f32")
+        out.append(p if out_fmt == "f32" else round_to(p, out_fmt))
+    return out

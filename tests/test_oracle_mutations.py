@@ -15,6 +15,8 @@ import pytest
 import oracle
 import test_oracle as pins  # noqa: E402  (tests/ is on sys.path under pytest)
 import test_oracle_double_quant as dq_pins  # noqa: E402
+import test_oracle_8bit as q8_pins  # noqa: E402
+import test_oracle_embedding as emb_pins  # noqa: E402
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "bnb4_oracle.c")
 
@@ -48,6 +50,21 @@ MUTATIONS = {
                                           "if (i == g0)\n                s = absmax[i];"),
     "dequant_absmax_other_rounding_order": ("out[i] = (float)q[i] * step;",
                                             "out[i] = (float)q[i] * scales[i / group] / 255.0f;"),
+    # the mistake the pages report: the normalised value snapped to a 65536-point grid
+    "quantize_8bit_snaps_to_grid": ("q[i] = (uint8_t)nearest_code8(v, code);",
+                                    "q[i] = (uint8_t)nearest_code8((float)(nearbyint(((double)v + 1.0) * 32767.5)"
+                                    " / 32767.5 - 1.0), code);"),
+    "quantize_8bit_ties_to_largest": ("if (dist < best_d) {", "if (dist <= best_d) {"),
+    "quantize_8bit_absmax_without_abs": ("const float mag = fabsf(load_elem(x, dtype, i));",
+                                         "const float mag = load_elem(x, dtype, i);"),
+    "dequantize_8bit_skips_fp32_rounding": (
+        "store_elem(out, out_dtype, i, entry * scale);",
+        "if (out_dtype == ORACLE_BF16) ((uint16_t *)out)[i] = encode_format(round_to_format("
+        "(double)entry * (double)scale, 8, -126, ldexp(2.0 - ldexp(1.0, -7), 127)), 7, 127, -126, 255);"
+        " else store_elem(out, out_dtype, i, entry * scale);"),
+    "embedding_rows_transposed": ("const int64_t e = idx[r] * D + k;", "const int64_t e = k * V + idx[r];"),
+    "embedding_rows_in_reverse_order": ("store_elem(out, out_dtype, r * D + k,",
+                                        "store_elem(out, out_dtype, (n_idx - 1 - r) * D + k,"),
 }
 
 PIN_CHECKS = [
@@ -66,6 +83,13 @@ PIN_CHECKS = [
     lambda: [dq_pins.test_double_quant_matches_exact_rationals(g) for g in (4, 7, 256)],
     lambda: dq_pins.test_double_quant_closed_forms(),
     lambda: dq_pins.test_double_quant_special_values(),
+    lambda: [q8_pins.test_matches_exact_rationals(k, "f32", 65, 64) for k in ("uniform", "log")],
+    lambda: q8_pins.test_dyadic_linear_table_closed_form(),
+    lambda: [q8_pins.test_every_midpoint_neighbourhood(k) for k in ("uniform", "log")],
+    lambda: q8_pins.test_special_blocks(),
+    lambda: q8_pins.test_dequant_double_rounding(),
+    lambda: [emb_pins.test_matches_exact_rationals(q, D, B) for q in ("nf4", "fp4") for D, B in ((12, 4), (13, 4))],
+    lambda: emb_pins.test_index_checks(),
 ]
 
 
@@ -95,7 +119,8 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
                      "oracle_quantize", "oracle_dequantize", "oracle_matmul",
                      "oracle_matmul_entries", "oracle_matmul_backward",
                      "oracle_matmul_backward_entries", "oracle_double_quant",
-                     "oracle_dequant_absmax"):
+                     "oracle_dequant_absmax", "oracle_quantize_8bit", "oracle_dequantize_8bit",
+                     "oracle_embedding_4bit"):
             f, g = getattr(real, attr), getattr(mutant, attr)
             g.restype, g.argtypes = f.restype, f.argtypes
         monkeypatch.setattr(oracle, "_lib", mutant)
@@ -103,6 +128,6 @@ def test_pins_catch_planted_mistake(name, monkeypatch):
         for check in PIN_CHECKS:
             try:
                 check()
-            except (AssertionError, ValueError):
+            except (AssertionError, ValueError, pytest.fail.Exception):
                 caught += 1
         assert caught > 0, f"no pin caught mutation {name}"

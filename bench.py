@@ -163,6 +163,24 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+# ------------------------------------------------------ across the ranks
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time.  Every rank calls this at the same point, in
+    the same order (it is a collective when world > 1)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job rate per second: the units all ranks processed (each rank runs its
+    own batch of the same size) over the slowest rank's time for `steps` steps."""
+    return units_per_rank_step * steps * world / (ms / 1e3)
+
+
 # ----------------------------------------------------------------- our arm
 
 class Step:
@@ -271,11 +289,8 @@ def run_ours(args, rank, world, dev):
     t1.record(stream)
     torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
-    ms = t0.elapsed_time(t1)
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
     if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
         torch.distributed.barrier()
 
     # per-launch durations: the same graph, the events read after each replay
@@ -287,14 +302,14 @@ def run_ours(args, rank, world, dev):
     per_op_ms = [statistics.mean(st[i] for st in per_step) for i in range(len(calls))]
     del graph, graph_ev
     step_bytes = sum(b for _, b, _ in ops)
-    value = step_bytes * args.steps * world / (ms / 1e3) / 1e9
+    value = job_rate(step_bytes, args.steps, world, ms) / 1e9
 
     # the next rows beyond the step (double-quantized statistics), timed on their own
     next_rows = time_next_rows(step, dev, args.steps, hbm)
 
     # e2e: the same step through the public API from pinned host buffers; the step's
     # inputs go host->device and every output comes back device->host, every step
-    e2e = run_e2e(args, step, dev, stream)
+    e2e = run_e2e(args, step, dev, stream, world)
 
     if rank != 0:
         return None
@@ -412,8 +427,9 @@ def time_next_rows(step, dev, steps, hbm):
     return out
 
 
-def run_e2e(args, step, dev, stream):
-    """Same step, host buffers in and out through the public API (pinned memory)."""
+def run_e2e(args, step, dev, stream, world=1):
+    """Same step, host buffers in and out through the public API (pinned memory);
+    whole-job rate over the slowest rank (every rank calls this)."""
     import bit_blockwise_weight_b200 as bnb4
     h_x = step.x.cpu().pin_memory()
     h_gemv_x = [g[4].cpu().pin_memory() for g in step.gemv]
@@ -446,10 +462,10 @@ def run_e2e(args, step, dev, stream):
         one()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     step_bytes = sum(b for _, b, _ in step_ops())
-    return {"value": round(step_bytes * steps / (ms / 1e3) / 1e9, 2), "unit": "GB/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+    return {"value": round(job_rate(step_bytes, steps, world, ms) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world, "steps": steps,
             "ms_per_step": round(ms / steps, 3)}
 
 

@@ -306,6 +306,7 @@ def run_ours(args, rank, world, dev):
 
     # the next rows beyond the step (double-quantized statistics), timed on their own
     next_rows = time_next_rows(step, dev, args.steps, hbm)
+    next_rows.update(time_8bit_and_embedding(dev, min(args.steps, 10), hbm))
 
     # e2e: the same step through the public API from pinned host buffers; the step's
     # inputs go host->device and every output comes back device->host, every step
@@ -424,6 +425,69 @@ def time_next_rows(step, dev, steps, hbm):
             out[f"gemv_4bit_{K}x{N}"]["us"] / out[f"gemv_4bit_dq_{K}x{N}"]["us"], 3)
     out["note"] = ("L2 flushed before each op; median of the replays; each time includes the "
                    "few us of its two event nodes")
+    return out
+
+
+def code8_table(seed: int = 0):
+    """A seeded 256-entry table for the 8-bit rows: -1, 0, 1 and magnitudes spread
+    log-uniformly down to 2^-24 (a wide dynamic range), strictly ascending."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    vals = {-1.0, 0.0, 1.0}
+    while len(vals) < 256:
+        v = float(np.float32(rng.choice([-1.0, 1.0]) * 2.0 ** rng.uniform(-24.0, 0.0)))
+        if v == 0.0 or abs(v) >= 2.0 ** -24:
+            vals.add(v)
+    return torch.tensor(sorted(vals), dtype=torch.float32)
+
+
+def time_8bit_and_embedding(dev, reps, hbm):
+    """Rows f3 and f4 outside the step, L2 flushed before each op (median):
+    quantize_8bit / dequantize_8bit of 2^26 bf16 elements (B 64), and 4096
+    embedding lookups in a 128256 x 4096 NF4 table (B 64) to bf16."""
+    import bit_blockwise_weight_b200 as b
+    from bit_blockwise_weight_b200 import synthetic
+    d = str(dev)
+    n = 1 << 26
+    code = code8_table(0)
+    x = synthetic.roundtrip_tensor(n, 0, "bf16", device=d)
+    q = torch.empty(n, dtype=torch.uint8, device=dev)
+    a8 = torch.empty(n // BLOCK, dtype=torch.float32, device=dev)
+    y8 = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    V, D, T = 128256, 4096, 4096
+    w = synthetic.normal((V * D,), 7, 0.02, "f32", device=d)
+    ep, ea = b.quantize_4bit(w, BLOCK, "nf4")
+    del w
+    g = torch.Generator(device=d).manual_seed(11)
+    idx = torch.randint(0, V, (T,), generator=g, device=d, dtype=torch.int64)
+    eo = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
+    ops = [("quantize_8bit_2p26_bf16", 2 * n + n + 4 * (n // BLOCK),
+            lambda: b.bnb4_quantize_8bit(x.data_ptr(), q.data_ptr(), a8.data_ptr(), n, BLOCK, code.data_ptr(), 2,
+                                         torch.cuda.current_stream(dev).cuda_stream)),
+           ("dequantize_8bit_2p26_bf16", n + 4 * (n // BLOCK) + 2 * n,
+            lambda: b.bnb4_dequantize_8bit(q.data_ptr(), a8.data_ptr(), y8.data_ptr(), n, BLOCK, code.data_ptr(), 2,
+                                           torch.cuda.current_stream(dev).cuda_stream)),
+           ("embedding_4bit_4096_of_128256x4096", T * (D // 2 + 4 * (D // BLOCK)) + 8 * T + 2 * T * D,
+            lambda: b.embedding_4bit(ep, ea, V, D, idx, BLOCK, "nf4", out=eo))]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    for _, _, f in ops:
+        f()
+    torch.cuda.synchronize(dev)
+    times = [[] for _ in ops]
+    for _ in range(max(3, reps)):
+        for i, (_, _, f) in enumerate(ops):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            times[i].append(e0.elapsed_time(e1))
+    out = {}
+    for (nm, nbytes, _), t in zip(ops, times):
+        us = statistics.median(t) * 1e3
+        out[nm] = {"us": round(us, 2), "bytes": nbytes, "GB/s": round(nbytes / (us / 1e6) / 1e9, 1),
+                   "hbm_frac": round(nbytes / (us / 1e6) / 1e9 / hbm, 4)}
     return out
 
 

@@ -5,6 +5,7 @@ runs in the library's CUDA kernels):
 
 * ``bnb4_quantize``, ``bnb4_dequantize``, ``bnb4_gemv``, ``bnb4_gemm``,
   ``bnb4_gemm_backward``, ``bnb4_gemv_dq``, ``bnb4_double_quant``, ``bnb4_dequant_absmax``,
+  ``bnb4_quantize_8bit``, ``bnb4_dequantize_8bit``, ``bnb4_embedding_4bit``,
   ``bnb4_device_status``, ``bnb4_selftest_wait_timeout``: the C ABI of
   ``include/bnb4.h`` one to one (raw
   device pointers as ints, sizes, enums, a ``cudaStream_t`` as an int).
@@ -53,6 +54,9 @@ def _load() -> ctypes.CDLL:
         "bnb4_gemm": (I, [P, P, P, P, P, I64, I64, I64, I, I, I, P]),
         "bnb4_gemm_backward": (I, [P, P, P, P, I64, I64, I64, I, I, I, P]),
         "bnb4_gemv_dq": (I, [P, P, P, P, I, P, P, I64, I64, I, I, I, P]),
+        "bnb4_quantize_8bit": (I, [P, P, P, I64, I, P, I, P]),
+        "bnb4_dequantize_8bit": (I, [P, P, P, I64, I, P, I, P]),
+        "bnb4_embedding_4bit": (I, [P, P, I64, I64, I, I, P, I64, P, I, P]),
         "bnb4_double_quant": (I, [P, I64, I, P, P, P]),
         "bnb4_dequant_absmax": (I, [P, P, I64, I, P, P]),
         "bnb4_device_status": (I, [P]),
@@ -75,6 +79,9 @@ bnb4_gemv = _lib.bnb4_gemv
 bnb4_gemm = _lib.bnb4_gemm
 bnb4_gemm_backward = _lib.bnb4_gemm_backward
 bnb4_gemv_dq = _lib.bnb4_gemv_dq
+bnb4_quantize_8bit = _lib.bnb4_quantize_8bit
+bnb4_dequantize_8bit = _lib.bnb4_dequantize_8bit
+bnb4_embedding_4bit = _lib.bnb4_embedding_4bit
 bnb4_double_quant = _lib.bnb4_double_quant
 bnb4_dequant_absmax = _lib.bnb4_dequant_absmax
 bnb4_device_status = _lib.bnb4_device_status
@@ -242,6 +249,58 @@ def dequant_absmax(absmax_q, scales, group: int = 256, out=None, stream=None):
     _need_cuda(out)
     _check(bnb4_dequant_absmax(_ptr(absmax_q), _ptr(scales), n, group, _ptr(out), _stream(stream)),
            "bnb4_dequant_absmax")
+    return out
+
+
+def _host_code8(code):
+    torch = _torch()
+    c = torch.as_tensor(code, dtype=torch.float32).detach().to("cpu").contiguous().reshape(-1)
+    if c.numel() != 256:
+        raise ValueError("an 8-bit code table has 256 entries")
+    return c  # kept alive by the caller for the duration of the call
+
+
+def quantize_8bit(x, code, blocksize: int = 64, stream=None):
+    """x: f32/f16/bf16 CUDA tensor; code: 256 ascending entries (host).
+    -> (q uint8[n], absmax f32[ceil(n/B)])."""
+    torch = _torch()
+    _need_cuda(x)
+    c = _host_code8(code)
+    n = x.numel()
+    q = torch.empty(n, dtype=torch.uint8, device=x.device)
+    absmax = torch.empty((n + blocksize - 1) // blocksize, dtype=torch.float32, device=x.device)
+    _check(bnb4_quantize_8bit(_ptr(x), _ptr(q), _ptr(absmax), n, blocksize, c.data_ptr(), _dtype_code(x),
+                              _stream(stream)), "bnb4_quantize_8bit")
+    return q, absmax
+
+
+def dequantize_8bit(q, absmax, code, blocksize: int = 64, dtype=None, out=None, stream=None):
+    """-> out[n] of dtype (default bfloat16)."""
+    torch = _torch()
+    _need_cuda(q, absmax)
+    c = _host_code8(code)
+    n = q.numel()
+    if out is None:
+        out = torch.empty(n, dtype=dtype or torch.bfloat16, device=q.device)
+    _need_cuda(out)
+    _check(bnb4_dequantize_8bit(_ptr(q), _ptr(absmax), _ptr(out), n, blocksize, c.data_ptr(), _dtype_code(out),
+                                _stream(stream)), "bnb4_dequantize_8bit")
+    return out
+
+
+def embedding_4bit(packed, absmax, V: int, D: int, idx, blocksize: int = 64, quant_type="nf4",
+                   dtype=None, out=None, stream=None):
+    """Rows idx (int64 CUDA tensor) of a [V, D] table quantized by quantize_4bit -> [len(idx), D]."""
+    torch = _torch()
+    _need_cuda(packed, absmax, idx)
+    if idx.dtype != torch.int64:
+        raise TypeError("indices must be int64")
+    n_idx = idx.numel()
+    if out is None:
+        out = torch.empty(n_idx, D, dtype=dtype or torch.bfloat16, device=packed.device)
+    _need_cuda(out)
+    _check(bnb4_embedding_4bit(_ptr(packed), _ptr(absmax), V, D, blocksize, _qtype(quant_type), _ptr(idx), n_idx,
+                               _ptr(out), _dtype_code(out), _stream(stream)), "bnb4_embedding_4bit")
     return out
 
 

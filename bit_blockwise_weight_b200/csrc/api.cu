@@ -76,6 +76,8 @@ const char *bnb4_status_string(bnb4_status s) {
     case BNB4_ERR_QTYPE: return "quant type must be NF4 or FP4";
     case BNB4_ERR_CUDA: return "CUDA kernel launch failed";
     case BNB4_ERR_TIMEOUT: return "a bounded device-side wait timed out";
+    case BNB4_ERR_CODE: return "8-bit code table must be 256 strictly ascending entries in [-1, 1], each 0 or >= 2^-24";
+    case BNB4_ERR_INDEX: return "an embedding index was out of range";
     }
     return "unknown status";
 }
@@ -173,12 +175,55 @@ bnb4_status bnb4_dequant_absmax(const uint8_t *absmax_q, const float *scales, in
     return from_cuda(launch_dequant_absmax(absmax_q, scales, n, group, absmax, stream));
 }
 
+bnb4_status bnb4_quantize_8bit(const void *x, uint8_t *q, float *absmax, int64_t n, int blocksize,
+                               const float *code, bnb4_dtype dt, cudaStream_t stream) {
+    if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
+    if (!valid_dtype(dt)) return BNB4_ERR_DTYPE;
+    if (n < 0 || n >= ((int64_t)1 << 40)) return BNB4_ERR_SHAPE;
+    if (!code) return BNB4_ERR_NULL;
+    if (!code8_table_usable(code)) return BNB4_ERR_CODE;
+    if (n == 0) return BNB4_OK;
+    if (!x || !q || !absmax) return BNB4_ERR_NULL;
+    if (!aligned16(x) || !aligned16(q) || !aligned16(absmax)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_quantize_8bit(x, q, absmax, n, blocksize, code, dt, stream));
+}
+
+bnb4_status bnb4_dequantize_8bit(const uint8_t *q, const float *absmax, void *out, int64_t n, int blocksize,
+                                 const float *code, bnb4_dtype dt, cudaStream_t stream) {
+    if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
+    if (!valid_dtype(dt)) return BNB4_ERR_DTYPE;
+    if (n < 0 || n >= ((int64_t)1 << 40)) return BNB4_ERR_SHAPE;
+    if (!code) return BNB4_ERR_NULL;
+    if (!code8_table_usable(code)) return BNB4_ERR_CODE;
+    if (n == 0) return BNB4_OK;
+    if (!q || !absmax || !out) return BNB4_ERR_NULL;
+    if (!aligned16(q) || !aligned16(absmax) || !aligned16(out)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_dequantize_8bit(q, absmax, out, n, blocksize, code, dt, stream));
+}
+
+bnb4_status bnb4_embedding_4bit(const uint8_t *packed, const float *absmax, int64_t V, int64_t D, int blocksize,
+                                bnb4_quant_type qt, const int64_t *idx, int64_t n_idx, void *out,
+                                bnb4_dtype dt, cudaStream_t stream) {
+    if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
+    if (!valid_qtype(qt)) return BNB4_ERR_QTYPE;
+    if (!valid_dtype(dt)) return BNB4_ERR_DTYPE;
+    if (V < 0 || D < 1 || n_idx < 0 || V >= kMaxDim || D >= kMaxDim || n_idx >= kMaxDim ||
+        (double)V * (double)D >= 0x1p40 || (double)n_idx * (double)D >= 0x1p40)
+        return BNB4_ERR_SHAPE;
+    if (n_idx == 0) return BNB4_OK;
+    if (!packed || !absmax || !idx || !out) return BNB4_ERR_NULL;
+    if (!aligned16(packed) || !aligned16(absmax) || !aligned16(idx) || !aligned16(out)) return BNB4_ERR_ALIGN;
+    return from_cuda(launch_embedding_4bit(packed, absmax, V, D, blocksize, qt, idx, n_idx, out, dt, stream));
+}
+
 bnb4_status bnb4_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return BNB4_ERR_CUDA;
-    unsigned int a = 0, b = 0;
-    if (gemm_tc_take_timeouts(&a) != cudaSuccess || gemm_small_take_timeouts(&b) != cudaSuccess)
+    unsigned int a = 0, b = 0, c = 0;
+    if (gemm_tc_take_timeouts(&a) != cudaSuccess || gemm_small_take_timeouts(&b) != cudaSuccess ||
+        quant_take_bad_indices(&c) != cudaSuccess)
         return BNB4_ERR_CUDA;
-    return (a != 0 || b != 0) ? BNB4_ERR_TIMEOUT : BNB4_OK;
+    if (a != 0 || b != 0) return BNB4_ERR_TIMEOUT;
+    return c != 0 ? BNB4_ERR_INDEX : BNB4_OK;
 }
 
 bnb4_status bnb4_selftest_wait_timeout(cudaStream_t stream) {

@@ -51,6 +51,21 @@ cudaError_t launch_double_quant(const float *absmax, int64_t n, int group, uint8
 cudaError_t launch_dequant_absmax(const uint8_t *q, const float *scales, int64_t n, int group, float *out,
                                   cudaStream_t stream);
 
+// 8-bit blockwise quantization against a caller's 256-entry table (host
+// pointer; code8_table_usable must hold)
+bool code8_table_usable(const float *code);
+cudaError_t launch_quantize_8bit(const void *x, uint8_t *q, float *absmax, int64_t n, int blocksize,
+                                 const float *code, bnb4_dtype dt, cudaStream_t stream);
+cudaError_t launch_dequantize_8bit(const uint8_t *q, const float *absmax, void *out, int64_t n, int blocksize,
+                                   const float *code, bnb4_dtype dt, cudaStream_t stream);
+
+// rows of a 4-bit-quantized [V, D] table; bad indices give zero rows and are
+// counted (quant_take_bad_indices reads and clears the count)
+cudaError_t launch_embedding_4bit(const uint8_t *packed, const float *absmax, int64_t V, int64_t D, int blocksize,
+                                  bnb4_quant_type qt, const int64_t *idx, int64_t n_idx, void *out,
+                                  bnb4_dtype dt, cudaStream_t stream);
+cudaError_t quant_take_bad_indices(unsigned int *count);
+
 // read and clear the count of bounded waits that gave up, per kernel file
 cudaError_t gemm_tc_take_timeouts(unsigned int *count);
 cudaError_t gemm_small_take_timeouts(unsigned int *count);

@@ -23,6 +23,11 @@
  *                       double_quant_block=256), dequant_absmax).
  *   bnb4_gemv_dq        gemv_4bit whose weight carries the double-quantized
  *                       absmax of the same section (8-bit statistics).
+ *   bnb4_quantize_8bit, "Feat/mps gemm 4bit bf16", What runs natively now
+ *   bnb4_dequantize_8bit (quantize_blockwise / dequantize_blockwise) and
+ *                       Correctness (exact nearest code, no lookup-table snap).
+ *   bnb4_embedding_4bit "mps-bitsandbytes 0.4.7", Quantized Embeddings
+ *                       (Embedding4bit: rows of a 4-bit-quantized table).
  *
  * Numeric contract (the readings of the pages that the CPU oracle follows):
  *   - absmax[b] = max |x_i| over block b, in fp32; blocks are `blocksize`
@@ -92,7 +97,9 @@ typedef enum {
     BNB4_ERR_DTYPE = 5,     /* dtype not accepted by this call                */
     BNB4_ERR_QTYPE = 6,     /* quant type not NF4 / FP4                       */
     BNB4_ERR_CUDA = 7,      /* a kernel launch failed                         */
-    BNB4_ERR_TIMEOUT = 8    /* a bounded device-side wait gave up             */
+    BNB4_ERR_TIMEOUT = 8,   /* a bounded device-side wait gave up             */
+    BNB4_ERR_CODE = 9,      /* an 8-bit code table that is not usable         */
+    BNB4_ERR_INDEX = 10     /* a lookup index was out of range (device side)  */
 } bnb4_status;
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
@@ -205,6 +212,49 @@ bnb4_status bnb4_dequant_absmax(const uint8_t *absmax_q, const float *scales,
                                 cudaStream_t stream);
 
 /*
+ * 8-bit blockwise quantization against the caller's code table (the pages
+ * print no 8-bit table).  Per block of `blocksize` elements (the last may be
+ * short): absmax = max |x| (fp32), v = x / absmax (IEEE fp32, 0 for an
+ * all-zero block), q[i] = the index of the entry nearest v, ties to the
+ * smaller index (exact; NaN gives 0), one byte per element.
+ *   x      [n] of x_dtype (f32 / f16 / bf16), 16-byte aligned.
+ *   q      [n] bytes out, absmax [ceil(n/blocksize)] float32 out; 16-byte aligned.
+ *   code   HOST pointer to 256 float32 entries, read during the call only:
+ *          strictly ascending, finite, in [-1, 1], each 0 or at least 2^-24
+ *          in magnitude (BNB4_ERR_CODE otherwise).
+ *   blocksize in {64, ..., 4096}; n >= 0.
+ */
+bnb4_status bnb4_quantize_8bit(const void *x, uint8_t *q, float *absmax,
+                               int64_t n, int blocksize, const float *code,
+                               bnb4_dtype x_dtype, cudaStream_t stream);
+
+/*
+ * Inverse: out[i] = RN_out_dtype(fp32(code[q[i]] * absmax[i / blocksize])).
+ * Same arguments and constraints (out [n] of out_dtype, 16-byte aligned).
+ */
+bnb4_status bnb4_dequantize_8bit(const uint8_t *q, const float *absmax,
+                                 void *out, int64_t n, int blocksize,
+                                 const float *code, bnb4_dtype out_dtype,
+                                 cudaStream_t stream);
+
+/*
+ * 4-bit embedding lookup.  The [V, D] table was quantized by bnb4_quantize as
+ * one flat array of V*D elements; out[r, k] = the dequantized element
+ * idx[r] * D + k (as bnb4_dequantize computes it), in out_dtype.
+ *   packed [ceil(V*D/2)], absmax [ceil(V*D/blocksize)], idx [n_idx] int64
+ *   (device), out [n_idx, D]; all 16-byte aligned.  V >= 0, D >= 1,
+ *   n_idx >= 0.  Rows with D % 16 == 0 take the vector path.
+ *   The indices are on the device and are not checked before the launch: an
+ *   index outside [0, V) gives a row of zeros and is counted, and the next
+ *   bnb4_device_status returns BNB4_ERR_INDEX.
+ */
+bnb4_status bnb4_embedding_4bit(const uint8_t *packed, const float *absmax,
+                                int64_t V, int64_t D, int blocksize,
+                                bnb4_quant_type quant_type, const int64_t *idx,
+                                int64_t n_idx, void *out, bnb4_dtype out_dtype,
+                                cudaStream_t stream);
+
+/*
  * Device-side status of the library's kernels (no counterpart on the pages:
  * a diagnostic for the bounded waits of the tensor-core kernels).  Every
  * mbarrier wait in those kernels gives up after about one second; a kernel
@@ -212,9 +262,10 @@ bnb4_status bnb4_dequant_absmax(const uint8_t *absmax_q, const float *scales,
  * undefined), frees its tensor memory and returns.
  * Synchronises `stream` (blocking the host), then reads and clears the
  * count of waits that gave up on the current device since the last call.
- * Returns BNB4_ERR_TIMEOUT if any did, BNB4_ERR_CUDA if the synchronisation
- * or the read failed (for instance after an earlier launch error), else
- * BNB4_OK.
+ * Returns BNB4_ERR_TIMEOUT if any did; else BNB4_ERR_INDEX if an embedding
+ * lookup met an index out of range since the last call (that count is read
+ * and cleared too); BNB4_ERR_CUDA if the synchronisation or a read failed
+ * (for instance after an earlier launch error); else BNB4_OK.
  */
 bnb4_status bnb4_device_status(cudaStream_t stream);
 

@@ -40,8 +40,8 @@ def test_library_exports_every_declared_symbol(name):
 
 def test_status_strings_and_version():
     assert bnb4.bnb4_version() >= 10000
-    for s in range(9):
-        assert bnb4.status_string(s)
+    for s in range(11):
+        assert bnb4.status_string(s) != "unknown status"
     assert bnb4.status_string(0) == "ok"
     assert bnb4.status_string(99) == "unknown status"
 
@@ -84,6 +84,47 @@ def test_matmul_argument_checks():
     b = bnb4.bnb4_gemm_backward
     assert b(A, A, A, A, 4, 128, 100, 64, 0, 2, None) == 4
     assert b(A, A, A, None, 4, 128, 128, 64, 0, 2, None) == 1
+
+
+def _code(values):
+    import numpy as np
+    c = np.ascontiguousarray(values, np.float32)
+    return c, c.ctypes.data
+
+
+def test_8bit_argument_checks():
+    import numpy as np
+    good, gp = _code((np.arange(256) - 128) / 128.0)
+    for bad_vals in (np.arange(256)[::-1] / 255.0,                          # descending
+                     np.where(np.arange(256) == 0, 2.0, np.linspace(-1, 1, 256)),   # out of range
+                     np.where(np.arange(256) == 128, 1e-30, (np.arange(256) - 128) / 128.0),  # tiny entry
+                     np.where(np.arange(256) == 5, np.nan, np.linspace(-1, 1, 256))):
+        bad, bp = _code(bad_vals)
+        assert bnb4.bnb4_quantize_8bit(A, A, A, 10, 64, bp, 0, None) == 9
+        assert bnb4.bnb4_dequantize_8bit(A, A, A, 10, 64, bp, 2, None) == 9
+    q = bnb4.bnb4_quantize_8bit
+    assert q(A, A, A, 10, 64, None, 0, None) == 1        # no table
+    assert q(A, A, A, 10, 32, gp, 0, None) == 3
+    assert q(A, A, A, 10, 64, gp, 4, None) == 5
+    assert q(A, A, A, -3, 64, gp, 0, None) == 4
+    assert q(A, A + 1, A, 10, 64, gp, 0, None) == 2
+    assert q(None, None, None, 0, 64, gp, 0, None) == 0  # n == 0: nothing to do
+    d = bnb4.bnb4_dequantize_8bit
+    assert d(A, None, A, 10, 64, gp, 2, None) == 1
+    assert d(A, A, A + 8, 10, 64, gp, 2, None) == 2
+    assert good.size == 256
+
+
+def test_embedding_argument_checks():
+    e = bnb4.bnb4_embedding_4bit
+    assert e(A, A, 100, 64, 64, 0, A, 0, A, 2, None) == 0     # no indices: nothing to do
+    assert e(A, A, 100, 0, 64, 0, A, 5, A, 2, None) == 4      # D < 1
+    assert e(A, A, -1, 64, 64, 0, A, 5, A, 2, None) == 4      # V < 0
+    assert e(A, A, 100, 64, 48, 0, A, 5, A, 2, None) == 3
+    assert e(A, A, 100, 64, 64, 3, A, 5, A, 2, None) == 6
+    assert e(A, A, 100, 64, 64, 0, A, 5, A, 7, None) == 5
+    assert e(A, A, 100, 64, 64, 0, None, 5, A, 2, None) == 1
+    assert e(A, A, 100, 64, 64, 0, A + 8, 5, A, 2, None) == 2
 
 
 def test_product_package_does_not_use_the_oracle():

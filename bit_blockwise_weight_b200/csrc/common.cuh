@@ -171,6 +171,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
 
+// The current device's index for per-device host caches (function attributes
+// are set per device context); 0 if it cannot be read or is 64 or above.
+inline int cache_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) d = 0;
+    return d;
+}
+
 // RN(s / 255) in fp32 (the step of a double-quantized absmax) without a
 // divide: Markstein's correction (P. Markstein, "Computation of elementary
 // functions on the IBM RISC System/6000 processor", 1990): with y = RN(1/255)

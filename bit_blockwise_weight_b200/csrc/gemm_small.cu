@@ -309,11 +309,12 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 template <typename D, int NT>
 cudaError_t set_smem_attr() {
-    static std::atomic<bool> done{false};
-    if (done.load(std::memory_order_relaxed)) return cudaSuccess;
+    static std::atomic<bool> done[64];  // per device: attributes belong to a device's context
+    const int dev = cache_device();
+    if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(gemm_small_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
-    if (e == cudaSuccess) done.store(true, std::memory_order_relaxed);
+    if (e == cudaSuccess) done[dev].store(true, std::memory_order_relaxed);
     return e;
 }
 

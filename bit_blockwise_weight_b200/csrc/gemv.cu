@@ -41,6 +41,8 @@
 // inverse of the double quantization gives, so the product is the plain
 // gemv's with that absmax.  The weight stream shrinks from 4.5 to about 4.13
 // bits per weight at blocks of 64.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -315,12 +317,17 @@ cudaError_t launch_t(const void *x, const uint8_t *W, const void *absmax, const 
     const int G = device_sm_count();
     const int kpad = ((K + 31) / 32) * 32;
     const size_t smem = kLut + (size_t)kWarps * STAGES * kSlot + kMaxRows * 4 + kWarps * 8 * 4 + (size_t)kpad * 2;
-    static int smem_set = 0;  // largest dynamic shared memory size set so far
-    if ((int)smem > smem_set) {
+    // the limit for the largest K, set once per device (attributes belong to a
+    // device's context); every launch asks for no more than that
+    constexpr size_t kSmemMax = kLut + (size_t)kWarps * STAGES * kSlot + kMaxRows * 4 + kWarps * 8 * 4 + kMaxK * 2;
+    static_assert(kSmemMax <= 227 * 1024, "shared memory plan at the largest K");
+    static std::atomic<bool> set[64];
+    const int dev = cache_device();
+    if (!set[dev].load(std::memory_order_relaxed)) {
         cudaError_t e = cudaFuncSetAttribute(gemv_kernel<D, DQ>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemMax);
         if (e != cudaSuccess) return e;
-        smem_set = (int)smem;
+        set[dev].store(true, std::memory_order_relaxed);
     }
     gemv_kernel<D, DQ><<<G, kThreads, smem, stream>>>(
         static_cast<const uint16_t *>(x), W, absmax, scales, log2G, static_cast<const uint16_t *>(bias),

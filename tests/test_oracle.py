@@ -262,12 +262,22 @@ def test_matmul_constant_blocks_closed_form():
 
 @pytest.mark.parametrize("qtype", ["nf4", "fp4"])
 def test_matmul_and_backward_exact_bruteforce(qtype):
+    _matmul_and_backward_exact(qtype, "bf16")
+
+
+@pytest.mark.parametrize("qtype", ["nf4", "fp4"])
+def test_matmul_and_backward_exact_bruteforce_fp32_activations(qtype):
+    """The fp32 compute dtype: fp32 activations, bias and gradients."""
+    _matmul_and_backward_exact(qtype, "f32")
+
+
+def _matmul_and_backward_exact(qtype, dt):
     M, N, K, B = 3, 64, 128, 64
     packed, absmax = _quant_weight(N, K, B, qtype, seed=5)
-    X = synthetic.activations(M, K, seed=6, dtype="bf16")
+    X = synthetic.activations(M, K, seed=6, dtype=dt)
     Xs = synthetic.storage_numpy(X).reshape(-1)
-    bias = synthetic.storage_numpy(synthetic.bias(N, seed=8, dtype="bf16"))
-    dY = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=9, dtype="bf16")).reshape(-1)
+    bias = synthetic.storage_numpy(synthetic.bias(N, seed=8, dtype=dt))
+    dY = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=9, dtype=dt)).reshape(-1)
     # exact weights from the brute force
     idx = []
     for byte in packed.tolist():
@@ -275,29 +285,29 @@ def test_matmul_and_backward_exact_bruteforce(qtype):
     idx = idx[:N * K]
     wq = bf.dequantize(idx, [Fraction(float(a)) for a in absmax], B, qtype, "f32")
     W = [wq[j * K:(j + 1) * K] for j in range(N)]
-    Xf = [_to_fracs(Xs[m * K:(m + 1) * K], "bf16") for m in range(M)]
-    bfr = _to_fracs(bias, "bf16")
+    Xf = [_to_fracs(Xs[m * K:(m + 1) * K], dt) for m in range(M)]
+    bfr = _to_fracs(bias, dt)
     Yex = bf.matmul(Xf, W, bfr)
-    Y = oracle.matmul(Xs, "bf16", packed, absmax, bias, M, N, K, B, qtype)
+    Y = oracle.matmul(Xs, dt, packed, absmax, bias, M, N, K, B, qtype)
     for m in range(M):
         for j in range(N):
             assert abs(Y[m, j] - float(Yex[m][j])) <= 1e-12 * (1 + abs(float(Yex[m][j])))
     # backward: dX = dY @ W (reduction over N) -- exact, then the entries form
-    dYf = [_to_fracs(dY[m * N:(m + 1) * N], "bf16") for m in range(M)]
+    dYf = [_to_fracs(dY[m * N:(m + 1) * N], dt) for m in range(M)]
     WT = [[W[j][k] for j in range(N)] for k in range(K)]
     dXex = bf.matmul(dYf, WT)
-    dX = oracle.matmul_backward(dY, "bf16", packed, absmax, M, N, K, B, qtype)
+    dX = oracle.matmul_backward(dY, dt, packed, absmax, M, N, K, B, qtype)
     for m in range(M):
         for k in range(K):
             assert abs(dX[m, k] - float(dXex[m][k])) <= 1e-12 * (1 + abs(float(dXex[m][k])))
     ms = np.array([0, 2, 1, 2])
     ks = np.array([0, 127, 64, 5])
     assert np.array_equal(
-        oracle.matmul_backward_entries(dY, "bf16", packed, absmax, M, N, K, B, qtype, ms, ks),
+        oracle.matmul_backward_entries(dY, dt, packed, absmax, M, N, K, B, qtype, ms, ks),
         dX[ms, ks])
     js = np.array([63, 0, 17, 32])
     assert np.array_equal(
-        oracle.matmul_entries(Xs, "bf16", packed, absmax, bias, M, N, K, B, qtype, ms, js),
+        oracle.matmul_entries(Xs, dt, packed, absmax, bias, M, N, K, B, qtype, ms, js),
         Y[ms, js])
 
 

@@ -127,6 +127,24 @@ def test_embedding_argument_checks():
     assert e(A, A, 100, 64, 64, 0, A + 8, 5, A, 2, None) == 2
 
 
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/bnb4.h compiles as C99 with warnings as errors; a C client links
+    libbnb4.so and gets the documented host-side results."""
+    import shutil
+    import subprocess
+    cc = shutil.which("cc") or shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    lib = bnb4.library_path()
+    exe = tmp_path / "c_abi_check"
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe),
+                           lib, "-Wl,-rpath," + os.path.dirname(lib)])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert out.returncode == 0, out.stderr
+    assert "c abi ok" in out.stdout
+
+
 def test_product_package_does_not_use_the_oracle():
     """The product never imports, includes, links or loads anything under oracle/."""
     pkg = os.path.join(ROOT, "bit_blockwise_weight_b200")

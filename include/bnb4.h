@@ -57,16 +57,19 @@
  *   packedW  uint8 [N, K/2]           absmax  float32 [N, K/blocksize].
  *
  * Ownership and execution:
- *   - Every pointer is a device pointer owned by the caller.  The library
- *     allocates no memory and holds no per-call state.
+ *   - Every pointer is a device pointer owned by the caller, except the
+ *     8-bit code table (`code`, a host pointer read during the call).  The
+ *     library allocates no memory and holds no per-call state.
  *   - Every call is asynchronous on `stream` (0 = the legacy default stream)
- *     and never synchronises the host.  Inputs must stay valid, and outputs
- *     must not be read, until work enqueued on `stream` has completed.
+ *     and never synchronises the host, except bnb4_device_status, whose job
+ *     that is.  Inputs must stay valid, and outputs must not be read, until
+ *     work enqueued on `stream` has completed.
  *   - Calls on different streams may run concurrently on disjoint outputs.
  *
  * Errors: each call returns a bnb4_status.  Argument checks happen on the
  * host before anything is enqueued; on any error nothing is enqueued and no
- * output is touched.  BNB4_ERR_CUDA reports a launch failure (the CUDA error
+ * output is touched.  The one device-side check (embedding indices, which
+ * live on the device) is reported by bnb4_device_status.  BNB4_ERR_CUDA reports a launch failure (the CUDA error
  * is left for the caller's next cudaGetLastError / synchronisation).  No call
  * ever falls back to another implementation.
  */

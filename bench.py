@@ -181,6 +181,37 @@ def job_rate(units_per_rank_step: float, steps: int, world: int, ms: float) -> f
     return units_per_rank_step * steps * world / (ms / 1e3)
 
 
+def roofline_and_parts(ops, per_op_ms, hbm, tc_sust, peak_kind, traffic=None):
+    """The roofline object for the op with the largest time share (HBM GB/s, or
+    TFLOP/s for the tensor-core matmuls) and the per-op breakdown.
+    ops: (name, algorithmic bytes, flops) per launch; per_op_ms: mean durations."""
+    traffic = traffic or profiled_traffic
+    di = max(range(len(per_op_ms)), key=lambda i: per_op_ms[i])
+    name, nbytes, nflops = ops[di]
+    if nflops and "_M512_" in name:
+        achieved = nflops / (per_op_ms[di] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_sust,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_sust, 4),
+                "traffic": traffic(name), "kernel": name,
+                "peak_kind": f"{peak_kind} sustained bf16"}
+    else:
+        achieved = nbytes / (per_op_ms[di] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4), "traffic": traffic(name),
+                "kernel": name, "peak_kind": f"{peak_kind} HBM copy"}
+    parts = {}
+    total = sum(per_op_ms)
+    for (nm, nb, nf), t in zip(ops, per_op_ms):
+        e = {"us": round(t * 1e3, 2), "GB/s": round(nb / (t / 1e3) / 1e9, 1),
+             "hbm_frac": round(nb / (t / 1e3) / 1e9 / hbm, 4),
+             "share": round(t / total, 4)}
+        if "_M512_" in nm:
+            e["TFLOP/s"] = round(nf / (t / 1e3) / 1e12, 1)
+            e["tensor_frac"] = round(nf / (t / 1e3) / 1e12 / tc_sust, 4)
+        parts[nm] = e
+    return roof, parts
+
+
 # ----------------------------------------------------------------- our arm
 
 class Step:
@@ -314,30 +345,7 @@ def run_ours(args, rank, world, dev):
 
     if rank != 0:
         return None
-    # dominant kernel by time share
-    shares = sorted(((t, i) for i, t in enumerate(per_op_ms)), reverse=True)
-    _, di = shares[0]
-    name, nbytes, nflops = ops[di]
-    if nflops and "_M512_" in name:
-        achieved = nflops / (per_op_ms[di] / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_sust,
-                "unit": "TFLOP/s", "frac": round(achieved / tc_sust, 4),
-                "traffic": profiled_traffic(name), "kernel": name,
-                "peak_kind": f"{peak_kind} sustained bf16"}
-    else:
-        achieved = nbytes / (per_op_ms[di] / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(achieved / hbm, 4), "traffic": profiled_traffic(name),
-                "kernel": name, "peak_kind": f"{peak_kind} HBM copy"}
-    parts = {}
-    for (nm, nb, nf), t in zip(ops, per_op_ms):
-        e = {"us": round(t * 1e3, 2), "GB/s": round(nb / (t / 1e3) / 1e9, 1),
-             "hbm_frac": round(nb / (t / 1e3) / 1e9 / hbm, 4),
-             "share": round(t / sum(per_op_ms), 4)}
-        if "_M512_" in nm:
-            e["TFLOP/s"] = round(nf / (t / 1e3) / 1e12, 1)
-            e["tensor_frac"] = round(nf / (t / 1e3) / 1e12 / tc_sust, 4)
-        parts[nm] = e
+    roof, parts = roofline_and_parts(ops, per_op_ms, hbm, tc_sust, peak_kind)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),

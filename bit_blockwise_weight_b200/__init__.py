@@ -11,9 +11,11 @@ runs in the library's CUDA kernels):
   device pointers as ints, sizes, enums, a ``cudaStream_t`` as an int).
   They return the integer status.
 * ``quantize_4bit``, ``dequantize_4bit``, ``gemv_4bit``, ``gemm_4bit``,
-  ``gemm_4bit_backward``: take torch CUDA tensors, allocate outputs with
-  torch, call the C ABI on the current stream and raise ``Bnb4Error`` on a
-  non-OK status.
+  ``gemm_4bit_backward``, ``double_quant``, ``dequant_absmax``,
+  ``gemv_4bit_dq``, ``quantize_8bit``, ``dequantize_8bit``,
+  ``embedding_4bit``, ``device_status``: take torch CUDA tensors (the 8-bit
+  code table on the host), allocate outputs with torch, call the C ABI on the
+  current stream and raise ``Bnb4Error`` on a non-OK status.
 
 Importing the package loads the shared library and fails loudly if it is
 missing.  There is no CPU or pure-PyTorch fallback.

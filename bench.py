@@ -111,7 +111,7 @@ def src_of(op):
 
 class ClockSampler:
     """SM clock and throttle reasons sampled through NVML every few ms while the
-    timed region runs (falls back to `nvidia-smi -lms` if NVML is unavailable)."""
+    timed region runs; stop() returns None when NVML cannot be used."""
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
 
@@ -219,7 +219,7 @@ class Step:
 
     def __init__(self, dev, seed):
         import bit_blockwise_weight_b200 as bnb4
-        from bit_blockwise_weight_b200 import synthetic
+        import synthetic
         self.bnb4 = bnb4
         d = str(dev)
         self.x = synthetic.roundtrip_tensor(N_ELEMS, seed, "bf16", device=d)
@@ -351,14 +351,10 @@ def run_ours(args, rank, world, dev):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) / N(0,0.02) tensors; no checkpoints)",
-        "config": {"workload": WORKLOAD, "n_elems": N_ELEMS, "quant_type": "nf4",
-                   "blocksize": BLOCK, "gemv_shapes_KN": GEMV_SHAPES,
-                   "smallm": {"M": SMALLM_M, "shapes_KN": SMALLM_SHAPES},
-                   "prefill_MKN": PREFILL, "parallelism": f"dp{world} (independent batches)",
-                   "l2": "inputs larger than L2 (step working set ~1.6 GB vs 126 MB L2)",
-                   "timing": "step captured once as a CUDA graph of its launches; K replays "
-                             "between two events; per-launch times from a second graph with an "
-                             "event node after each launch"},
+        "config": bench_config(world),
+        "timing": "step captured once as a CUDA graph of its launches; K replays between two "
+                  "events; per-launch times from a second graph with an event node after each "
+                  "launch",
         "roofline": roof,
         "parts": parts,
         "next_rows": next_rows,
@@ -368,7 +364,7 @@ def run_ours(args, rank, world, dev):
         "library": bnb4.library_path(),
     }
     if args.cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        line["cpu_baseline"] = cpu_baseline()
     return line
 
 
@@ -454,7 +450,7 @@ def time_8bit_and_embedding(dev, reps, hbm):
     quantize_8bit / dequantize_8bit of 2^26 bf16 elements (B 64), and 4096
     embedding lookups in a 128256 x 4096 NF4 table (B 64) to bf16."""
     import bit_blockwise_weight_b200 as b
-    from bit_blockwise_weight_b200 import synthetic
+    import synthetic
     d = str(dev)
     n = 1 << 26
     code = code8_table(0)
@@ -543,22 +539,23 @@ def run_e2e(args, step, dev, stream, world=1):
 
 # ------------------------------------------------------------ CPU oracle arm
 
-def oracle_sample(seconds_budget: float):
+def oracle_sample(seed: int = 0):
     """Time the CPU oracle on a bounded sample of every op of the step.
 
-    Returns (extrapolated GB/s for the whole step, description, per-op detail).
-    Each op runs on a slice of its workload (a number of elements, rows or
-    output entries); its time is scaled to the full op by that fraction.
+    Returns (extrapolated GB/s for the whole step, extrapolated seconds per
+    step, per-op detail).  Each op runs on a slice of its workload (a number
+    of elements, rows or output entries); its time is scaled to the full op
+    by that fraction.  `seed` picks the slice's inputs.
     """
     import numpy as np
     import oracle
-    from bit_blockwise_weight_b200 import synthetic
+    import synthetic
     oracle.lib()
     ops = step_ops()
     detail = {}
     full_time = 0.0
     frac_q = 1 << 24
-    x = synthetic.storage_numpy(synthetic.roundtrip_tensor(frac_q, 0, "bf16"))
+    x = synthetic.storage_numpy(synthetic.roundtrip_tensor(frac_q, seed, "bf16"))
     t = time.perf_counter()
     p, a = oracle.quantize(x, "bf16", BLOCK, "nf4")
     tq = (time.perf_counter() - t) * (N_ELEMS / frac_q)
@@ -570,7 +567,7 @@ def oracle_sample(seconds_budget: float):
     full_time += tq + td
 
     def mm_rows(K, N, M, rows, backward=False):
-        w = synthetic.weight(min(N, 64), K, 0).numpy().reshape(-1)
+        w = synthetic.weight(min(N, 64), K, seed).numpy().reshape(-1)
         wp, wa = oracle.quantize(w, "f32", BLOCK, "nf4")
         Nw = min(N, 64)
         if backward:
@@ -603,35 +600,54 @@ def oracle_sample(seconds_budget: float):
     return step_bytes / full_time / 1e9, full_time, detail
 
 
-def cpu_baseline(seconds):
-    gbs, full_s, detail = oracle_sample(seconds)
-    return {"value": round(gbs, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": ("single-threaded C oracle on slices of every op (2^24 quantize/"
-                       "dequantize elements, 2048-16384 output entries per matmul), scaled to the "
-                       f"full step: {round(full_s, 1)} s per step extrapolated"),
+def oracle_all_cores(threads=None):
+    """The oracle on every host core at once: one thread per core, each timing
+    its own slice of every op (the C oracle runs through ctypes, which releases
+    the GIL for the call).  Returns (whole-step GB/s over all threads, threads,
+    mean extrapolated seconds per step and thread)."""
+    import concurrent.futures as cf
+    threads = threads or os.cpu_count() or 1
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        res = list(ex.map(oracle_sample, range(threads)))
+    per_thread_s = statistics.mean(r[1] for r in res)
+    step_bytes = sum(b for _, b, _ in step_ops())
+    return threads * step_bytes / per_thread_s / 1e9, threads, per_thread_s
+
+
+def cpu_baseline(measured=None):
+    gbs, threads, per_thread_s = measured or oracle_all_cores()
+    return {"value": round(gbs, 6), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": (f"the C oracle on {threads} host threads at once (one per core), each on its "
+                       "own slice of every op of the step (2^24 quantize/dequantize elements, "
+                       "2048-16384 output entries per matmul), each slice's time scaled to the "
+                       f"full step ({round(per_thread_s, 1)} s per step and thread, extrapolated); "
+                       "value = all threads' steps over that time"),
             "host_nproc": os.cpu_count()}
 
 
+def bench_config(world):
+    return {"workload": WORKLOAD, "n_elems": N_ELEMS, "quant_type": "nf4",
+            "blocksize": BLOCK, "gemv_shapes_KN": GEMV_SHAPES,
+            "smallm": {"M": SMALLM_M, "shapes_KN": SMALLM_SHAPES},
+            "prefill_MKN": PREFILL, "parallelism": f"dp{world} (independent batches)",
+            "l2": "inputs larger than L2 (step working set ~1.6 GB vs 126 MB L2)"}
+
+
 def run_reference(args):
-    """The reference arm: the CPU oracle, timed on bounded samples of the workload."""
+    """The reference arm: the CPU oracle on every host core, timed on bounded
+    samples of the workload (one sample per step)."""
     for _ in range(args.warmup):
-        oracle_sample(1.0)
+        oracle_all_cores()
     t = time.perf_counter()
-    vals = []
-    for _ in range(args.steps):
-        gbs, full_s, _ = oracle_sample(1.0)
-        vals.append(gbs)
+    runs = [oracle_all_cores() for _ in range(args.steps)]
     wall = time.perf_counter() - t
-    v = statistics.mean(vals)
-    base = cpu_baseline(1.0)
-    base["value"] = round(v, 6)
+    v = statistics.mean(r[0] for r in runs)
+    base = cpu_baseline((v, runs[0][1], statistics.mean(r[2] for r in runs)))
     return {"metric": METRIC, "value": round(v, 6), "unit": "GB/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(wall / args.steps * 1e3, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference",
-            "config": {"workload": WORKLOAD, "n_elems": N_ELEMS, "quant_type": "nf4",
-                       "blocksize": BLOCK},
+            "impl": "reference", "config": bench_config(1),
             "cpu_baseline": base,
             "e2e": {"value": round(v, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -657,7 +673,7 @@ def profile_case(name):
     Setup launches (input draws, weight quantization) come first; the kernel of
     interest is the last launch of its kind."""
     import bit_blockwise_weight_b200 as bnb4
-    from bit_blockwise_weight_b200 import synthetic
+    import synthetic
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     d = str(dev)
@@ -698,7 +714,6 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
-    ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
                     help="run one launch of one kernel on a small case for an ncu capture "
                          "(prints no bench line)")

@@ -85,18 +85,15 @@ dequant_absmax_kernel(const uint8_t *__restrict__ q, const float *__restrict__ s
 }
 
 template <typename Kern>
-int persistent_grid(Kern kernel, std::atomic<int> (&cache)[64], int64_t work_ctas) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    int per_sm = cache[dev].load(std::memory_order_relaxed);
-    if (per_sm == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0) != cudaSuccess ||
-            per_sm <= 0) {
+int persistent_grid(Kern kernel, std::atomic<int> (&cache)[kMaxDevices], int64_t work_ctas) {
+    const int per_sm = cached_per_device(cache, [&] {
+        int v = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, kThreads, 0) != cudaSuccess || v <= 0) {
             (void)cudaGetLastError();
-            per_sm = 4;
+            v = 4;
         }
-        cache[dev].store(per_sm, std::memory_order_relaxed);
-    }
+        return v;
+    });
     int64_t g = (int64_t)device_sm_count() * per_sm;
     if (work_ctas < g) g = work_ctas;
     return (int)(g < 1 ? 1 : g);
@@ -106,7 +103,7 @@ int persistent_grid(Kern kernel, std::atomic<int> (&cache)[64], int64_t work_cta
 
 cudaError_t launch_double_quant(const float *absmax, int64_t n, int group, uint8_t *q, float *scales,
                                 cudaStream_t stream) {
-    static std::atomic<int> cache[64];
+    static std::atomic<int> cache[kMaxDevices];
     const int log2G = ilog2(group);
     const int64_t ngroups = (n + group - 1) / group;
     const int grid = persistent_grid(double_quant_kernel, cache, (ngroups + kWarps - 1) / kWarps);
@@ -116,7 +113,7 @@ cudaError_t launch_double_quant(const float *absmax, int64_t n, int group, uint8
 
 cudaError_t launch_dequant_absmax(const uint8_t *q, const float *scales, int64_t n, int group, float *out,
                                   cudaStream_t stream) {
-    static std::atomic<int> cache[64];
+    static std::atomic<int> cache[kMaxDevices];
     const int log2G = ilog2(group);
     const int grid = persistent_grid(dequant_absmax_kernel, cache, (n + kThreads * 4 - 1) / (kThreads * 4));
     dequant_absmax_kernel<<<grid, kThreads, 0, stream>>>(q, scales, n, log2G, out);

@@ -12,16 +12,16 @@
 namespace bnb4 {
 
 int device_sm_count() {
-    static std::atomic<int> cache[64];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    int v = cache[dev].load(std::memory_order_relaxed);
-    if (v == 0) {
-        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
-            v = 148;
-        cache[dev].store(v, std::memory_order_relaxed);
-    }
-    return v;
+    static std::atomic<int> cache[kMaxDevices];
+    return cached_per_device(cache, [] {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) {
+            (void)cudaGetLastError();
+            return 148;  // every grid here is correct for any size; this only sizes it
+        }
+        return v;
+    });
 }
 
 namespace {
@@ -56,6 +56,9 @@ bnb4_status check_matmul(const void *a, const uint8_t *W, const float *absmax, c
 
 bnb4_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA; }
 
+// reads and clears a device error count in one atomic exchange
+__global__ void take_counter_kernel(unsigned int *count) { (void)atomicExch(count, 0u); }
+
 }  // namespace
 }  // namespace bnb4
 
@@ -78,6 +81,7 @@ const char *bnb4_status_string(bnb4_status s) {
     case BNB4_ERR_TIMEOUT: return "a bounded device-side wait timed out";
     case BNB4_ERR_CODE: return "8-bit code table must be 256 strictly ascending entries in [-1, 1], each 0 or >= 2^-24";
     case BNB4_ERR_INDEX: return "an embedding index was out of range";
+    case BNB4_ERR_DEVICE: return "a kernel found its launch configuration unusable and wrote nothing";
     }
     return "unknown status";
 }
@@ -218,12 +222,30 @@ bnb4_status bnb4_embedding_4bit(const uint8_t *packed, const float *absmax, int6
 
 bnb4_status bnb4_device_status(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return BNB4_ERR_CUDA;
-    unsigned int a = 0, b = 0, c = 0;
-    if (gemm_tc_take_timeouts(&a) != cudaSuccess || gemm_small_take_timeouts(&b) != cudaSuccess ||
-        quant_take_bad_indices(&c) != cudaSuccess)
+    // in order of severity: the first nonzero count is the one reported, and
+    // only it is cleared; the others stay for the next call
+    unsigned int *w[4] = {nullptr, nullptr, nullptr, nullptr};
+    if (gemv_layout_errors_address(&w[0]) != cudaSuccess || gemm_tc_timeouts_address(&w[1]) != cudaSuccess ||
+        gemm_small_timeouts_address(&w[2]) != cudaSuccess || quant_bad_indices_address(&w[3]) != cudaSuccess)
         return BNB4_ERR_CUDA;
-    if (a != 0 || b != 0) return BNB4_ERR_TIMEOUT;
-    return c != 0 ? BNB4_ERR_INDEX : BNB4_OK;
+    const bnb4_status code[4] = {BNB4_ERR_DEVICE, BNB4_ERR_TIMEOUT, BNB4_ERR_TIMEOUT, BNB4_ERR_INDEX};
+    for (int i = 0; i < 4; ++i) {
+        unsigned int v = 0;
+        if (cudaMemcpy(&v, w[i], sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BNB4_ERR_CUDA;
+        if (v == 0) continue;
+        // one atomic exchange on the device: an increment that lands after the
+        // read above is taken with it, never lost
+        take_counter_kernel<<<1, 1, 0, stream>>>(w[i]);
+        if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess) return BNB4_ERR_CUDA;
+        // both timeout words are one status
+        if (i == 1) {
+            take_counter_kernel<<<1, 1, 0, stream>>>(w[2]);
+            if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
+                return BNB4_ERR_CUDA;
+        }
+        return code[i];
+    }
+    return BNB4_OK;
 }
 
 bnb4_status bnb4_selftest_wait_timeout(cudaStream_t stream) {

@@ -10,6 +10,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/bnb4.h"
 
 namespace bnb4 {
@@ -137,6 +139,7 @@ struct QuantTables {
     uint32_t key[32];
     uint32_t rank_lohi[32];
     int fast;
+    int valid;  // 0: a cell held two thresholds (the tables are unusable)
 };
 constexpr float kNear = 0x1p-19f;
 
@@ -171,12 +174,40 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v >> 1); }
 
-// The current device's index for per-device host caches (function attributes
-// are set per device context); 0 if it cannot be read or is 64 or above.
+// Per-device host caches (occupancy, SM counts, shared-memory attributes:
+// function attributes belong to a device's context) hold kMaxDevices slots.
+// cache_device() is the current device's slot, or -1 when the device cannot be
+// read or its index is kMaxDevices or above; callers then do the work the
+// cache would have saved on every call.
+constexpr int kMaxDevices = 64;
+
 inline int cache_device() {
     int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
     return d;
+}
+
+// cache[device] if set (nonzero), else compute() (stored when nonzero)
+template <typename F>
+int cached_per_device(std::atomic<int> (&cache)[kMaxDevices], F compute) {
+    const int d = cache_device();
+    if (d >= 0) {
+        const int v = cache[d].load(std::memory_order_relaxed);
+        if (v != 0) return v;
+    }
+    const int v = compute();
+    if (d >= 0 && v != 0) cache[d].store(v, std::memory_order_relaxed);
+    return v;
+}
+
+// calls set() once per device (every time when the device has no cache slot)
+template <typename F>
+cudaError_t once_per_device(std::atomic<bool> (&done)[kMaxDevices], F set) {
+    const int d = cache_device();
+    if (d >= 0 && done[d].load(std::memory_order_relaxed)) return cudaSuccess;
+    const cudaError_t e = set();
+    if (e == cudaSuccess && d >= 0) done[d].store(true, std::memory_order_relaxed);
+    return e;
 }
 
 // RN(s / 255) in fp32 (the step of a double-quantized absmax) without a

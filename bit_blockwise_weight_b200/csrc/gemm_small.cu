@@ -309,13 +309,10 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 template <typename D, int NT>
 cudaError_t set_smem_attr() {
-    static std::atomic<bool> done[64];  // per device: attributes belong to a device's context
-    const int dev = cache_device();
-    if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(gemm_small_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e == cudaSuccess) done[dev].store(true, std::memory_order_relaxed);
-    return e;
+    static std::atomic<bool> done[kMaxDevices];  // per device: attributes belong to a device's context
+    return once_per_device(done, [] {
+        return cudaFuncSetAttribute(gemm_small_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    });
 }
 
 cudaLaunchConfig_t make_cfg(dim3 grid, int S, cudaStream_t stream, cudaLaunchAttribute *attr) {
@@ -336,12 +333,9 @@ cudaLaunchConfig_t make_cfg(dim3 grid, int S, cudaStream_t stream, cudaLaunchAtt
 // CTAs in clusters of S (1, 2, 4, 8) resident at once on the current device
 template <typename D, int NT>
 int cluster_capacity(int S) {
-    static std::atomic<int> cache[64][4];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
-    const int si = S == 1 ? 0 : S == 2 ? 1 : S == 4 ? 2 : 3;
-    int v = cache[dev][si].load(std::memory_order_relaxed);
-    if (v == 0) {
+    static std::atomic<int> cache[4][kMaxDevices];
+    const int ci = S == 1 ? 0 : S == 2 ? 1 : S == 4 ? 2 : 3;
+    return cached_per_device(cache[ci], [&] {
         int n = 0;
         cudaLaunchAttribute attr[1];
         cudaLaunchConfig_t cfg = make_cfg(dim3(1, 1, S), S, 0, attr);
@@ -350,10 +344,8 @@ int cluster_capacity(int S) {
             (void)cudaGetLastError();
             n = device_sm_count() / S;
         }
-        v = n * S;
-        cache[dev][si].store(v, std::memory_order_relaxed);
-    }
-    return v;
+        return n * S;
+    });
 }
 
 // Row groups G and K split S.  A CTA's time is taken as its runs times
@@ -418,7 +410,7 @@ cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const
 
 }  // namespace
 
-cudaError_t gemm_small_take_timeouts(unsigned int *count) { return take_wait_timeouts(count); }
+cudaError_t gemm_small_timeouts_address(unsigned int **p) { return wait_timeouts_address(p); }
 
 cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
                               const void *bias, void *Y, int64_t M, int64_t N, int64_t K,

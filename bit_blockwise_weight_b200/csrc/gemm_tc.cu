@@ -457,13 +457,10 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 template <typename D, bool BWD, int BN>
 cudaError_t set_smem_attr() {
-    static std::atomic<bool> done[64];  // per device: attributes belong to a device's context
-    const int dev = cache_device();
-    if (done[dev].load(std::memory_order_relaxed)) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<D, BWD, BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    if (e == cudaSuccess) done[dev].store(true, std::memory_order_relaxed);
-    return e;
+    static std::atomic<bool> done[kMaxDevices];  // per device: attributes belong to a device's context
+    return once_per_device(done, [] {
+        return cudaFuncSetAttribute(gemm_tc_kernel<D, BWD, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    });
 }
 
 cudaLaunchConfig_t make_cfg(dim3 grid, int C, cudaStream_t stream, cudaLaunchAttribute *attr) {
@@ -486,12 +483,9 @@ cudaLaunchConfig_t make_cfg(dim3 grid, int C, cudaStream_t stream, cudaLaunchAtt
 // SM count.  Queried once per device and cluster size.
 template <typename D, bool BWD, int BN>
 int cluster_capacity(int C) {
-    static std::atomic<int> cache[64][4];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    static std::atomic<int> cache[4][kMaxDevices];
     const int ci = C == 1 ? 0 : C == 2 ? 1 : C == 4 ? 2 : 3;
-    int v = cache[dev][ci].load(std::memory_order_relaxed);
-    if (v == 0) {
+    return cached_per_device(cache[ci], [&] {
         int n = 0;
         cudaLaunchAttribute attr[1];
         cudaLaunchConfig_t cfg = make_cfg(dim3(1, 1, C), C, 0, attr);
@@ -500,10 +494,8 @@ int cluster_capacity(int C) {
             (void)cudaGetLastError();
             n = device_sm_count() / C;
         }
-        v = n * C;
-        cache[dev][ci].store(v, std::memory_order_relaxed);
-    }
-    return v;
+        return n * C;
+    });
 }
 
 template <typename D, bool BWD, int BN>
@@ -619,7 +611,7 @@ cudaError_t launch_selftest_wait_timeout(cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-cudaError_t gemm_tc_take_timeouts(unsigned int *count) { return take_wait_timeouts(count); }
+cudaError_t gemm_tc_timeouts_address(unsigned int **p) { return wait_timeouts_address(p); }
 
 cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax, const void *bias,
                            void *D, int64_t M, int64_t N, int64_t K, int blocksize,

@@ -60,15 +60,18 @@ cudaError_t launch_dequantize_8bit(const uint8_t *q, const float *absmax, void *
                                    const float *code, bnb4_dtype dt, cudaStream_t stream);
 
 // rows of a 4-bit-quantized [V, D] table; bad indices give zero rows and are
-// counted (quant_take_bad_indices reads and clears the count)
+// counted in a device word (quant_bad_indices_address)
 cudaError_t launch_embedding_4bit(const uint8_t *packed, const float *absmax, int64_t V, int64_t D, int blocksize,
                                   bnb4_quant_type qt, const int64_t *idx, int64_t n_idx, void *out,
                                   bnb4_dtype dt, cudaStream_t stream);
-cudaError_t quant_take_bad_indices(unsigned int *count);
+cudaError_t quant_bad_indices_address(unsigned int **p);
 
-// read and clear the count of bounded waits that gave up, per kernel file
-cudaError_t gemm_tc_take_timeouts(unsigned int *count);
-cudaError_t gemm_small_take_timeouts(unsigned int *count);
+// Device addresses (current device) of the words that count device-side
+// errors: gemv launches that found their shared-memory plan unusable (they
+// write nothing), and bounded waits that gave up, per kernel file
+cudaError_t gemv_layout_errors_address(unsigned int **p);
+cudaError_t gemm_tc_timeouts_address(unsigned int **p);
+cudaError_t gemm_small_timeouts_address(unsigned int **p);
 
 // one kernel whose mbarrier wait runs out after 1 ms (tests the timeout path)
 cudaError_t launch_selftest_wait_timeout(cudaStream_t stream);

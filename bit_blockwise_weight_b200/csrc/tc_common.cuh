@@ -235,12 +235,9 @@ __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity) {
 
 // ------------------------------------------------------------ host side
 
-// Read and clear this file's count of timed-out waits on the current device.
-inline cudaError_t take_wait_timeouts(unsigned int *count) {
-    cudaError_t e = cudaMemcpyFromSymbol(count, g_wait_timeouts, sizeof(unsigned int));
-    if (e != cudaSuccess) return e;
-    const unsigned int zero = 0;
-    return cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(unsigned int));
+// Device address of this file's count of timed-out waits on the current device.
+inline cudaError_t wait_timeouts_address(unsigned int **p) {
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(p), g_wait_timeouts);
 }
 
 
@@ -264,7 +261,9 @@ CUresult encode_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base,
     cuuint64_t strides[1] = {(cuuint64_t)pitch_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    return get_encode()(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode();
+    if (!encode) return CUDA_ERROR_NOT_SUPPORTED;
+    return encode(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }

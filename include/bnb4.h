@@ -68,8 +68,10 @@
  *
  * Errors: each call returns a bnb4_status.  Argument checks happen on the
  * host before anything is enqueued; on any error nothing is enqueued and no
- * output is touched.  The one device-side check (embedding indices, which
- * live on the device) is reported by bnb4_device_status.  BNB4_ERR_CUDA reports a launch failure (the CUDA error
+ * output is touched.  Checks that can only be made on the device (embedding
+ * indices, which live on the device; bounded waits; the gemv's shared-memory
+ * plan) are reported by bnb4_device_status.  BNB4_ERR_CUDA reports a launch
+ * failure (the CUDA error
  * is left for the caller's next cudaGetLastError / synchronisation).  No call
  * ever falls back to another implementation.
  */
@@ -102,7 +104,8 @@ typedef enum {
     BNB4_ERR_CUDA = 7,      /* a kernel launch failed                         */
     BNB4_ERR_TIMEOUT = 8,   /* a bounded device-side wait gave up             */
     BNB4_ERR_CODE = 9,      /* an 8-bit code table that is not usable         */
-    BNB4_ERR_INDEX = 10     /* a lookup index was out of range (device side)  */
+    BNB4_ERR_INDEX = 10,    /* a lookup index was out of range (device side)  */
+    BNB4_ERR_DEVICE = 11    /* a kernel found its launch unusable (device side) */
 } bnb4_status;
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
@@ -259,16 +262,25 @@ bnb4_status bnb4_embedding_4bit(const uint8_t *packed, const float *absmax,
 
 /*
  * Device-side status of the library's kernels (no counterpart on the pages:
- * a diagnostic for the bounded waits of the tensor-core kernels).  Every
- * mbarrier wait in those kernels gives up after about one second; a kernel
- * whose wait gave up skips its remaining work (its outputs are then
- * undefined), frees its tensor memory and returns.
- * Synchronises `stream` (blocking the host), then reads and clears the
- * count of waits that gave up on the current device since the last call.
- * Returns BNB4_ERR_TIMEOUT if any did; else BNB4_ERR_INDEX if an embedding
- * lookup met an index out of range since the last call (that count is read
- * and cleared too); BNB4_ERR_CUDA if the synchronisation or a read failed
- * (for instance after an earlier launch error); else BNB4_OK.
+ * a diagnostic for checks that can only happen on the device).  Three kinds
+ * of device-side error are counted, in device words shared by every stream
+ * of the current device:
+ *   BNB4_ERR_DEVICE   a gemv launch found that its shared-memory plan does not
+ *                     fit the memory it was given (it wrote nothing);
+ *   BNB4_ERR_TIMEOUT  a bounded mbarrier wait of a tensor-core kernel gave up
+ *                     after about one second (that kernel skipped its
+ *                     remaining work, so its outputs are undefined, freed its
+ *                     tensor memory and returned);
+ *   BNB4_ERR_INDEX    an embedding lookup met an index outside [0, V).
+ * Synchronises `stream` (blocking the host), then returns the most severe
+ * kind with a nonzero count, in the order above, and clears that count alone
+ * (one atomic exchange on the device, so an error raised meanwhile by a
+ * kernel on another stream is not lost); the other counts stay for the next
+ * call.  BNB4_OK when every count is zero; BNB4_ERR_CUDA if the
+ * synchronisation or a read failed (for instance after an earlier launch
+ * error).  The counts cover every kernel that finished before the call, on
+ * any stream; two host threads calling this at once may each see the other's
+ * report.
  */
 bnb4_status bnb4_device_status(cudaStream_t stream);
 

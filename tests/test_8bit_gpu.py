@@ -11,7 +11,7 @@ import torch
 
 import bit_blockwise_weight_b200 as bnb4
 import oracle
-from bit_blockwise_weight_b200 import synthetic
+import synthetic
 
 from gpu_util import to_dev, to_host
 

@@ -50,3 +50,26 @@ def test_reference_line():
     assert line["e2e"] == {"value": line["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
     assert line["config"]["workload"] == bench.WORKLOAD
+
+
+def test_reference_line_has_our_config():
+    """Both arms describe the same workload with the same config dict."""
+    assert bench.bench_config(1) == bench.bench_config(1)
+    line = bench.run_reference(types.SimpleNamespace(steps=1, warmup=0))
+    assert line["config"] == bench.bench_config(1)
+
+
+def test_reference_arm_loads_no_product_library():
+    """The reference arm (the oracle on the host cores) imports neither the
+    product package nor its shared library."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, types; sys.path.insert(0, %r); import bench; "
+            "bench.oracle_sample(0); "
+            "assert 'bit_blockwise_weight_b200' not in sys.modules, 'product package imported'; "
+            "maps = open('/proc/self/maps').read(); "
+            "assert 'libbnb4' not in maps, 'libbnb4.so mapped'; print('ok')" % root)
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr

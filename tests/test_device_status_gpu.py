@@ -39,3 +39,21 @@ def test_timed_out_wait_is_reported_once():
     p, a = bnb4.quantize_4bit(x, 64, "nf4")
     torch.cuda.synchronize()
     assert p.numel() == 2048 and a.numel() == 64
+
+
+INDEX = 10  # BNB4_ERR_INDEX
+
+
+def test_two_kinds_are_reported_one_after_the_other():
+    """A timed-out wait and a bad embedding index raised before one status
+    call: the more severe (timeout) is reported and cleared first, the index
+    report is kept for the next call, then all is clear."""
+    assert bnb4.device_status() == bnb4.STATUS_OK
+    w = torch.randn(64 * 128, device="cuda") * 0.02
+    p, a = bnb4.quantize_4bit(w, 64, "nf4")
+    idx = torch.tensor([0, 64, 3], dtype=torch.int64, device="cuda")   # 64 is out of range
+    bnb4.embedding_4bit(p, a, 64, 128, idx, 64, "nf4")
+    assert bnb4.bnb4_selftest_wait_timeout(_stream()) == bnb4.STATUS_OK
+    assert bnb4.device_status() == TIMEOUT
+    assert bnb4.device_status() == INDEX
+    assert bnb4.device_status() == bnb4.STATUS_OK

@@ -12,7 +12,7 @@ import torch
 
 import bit_blockwise_weight_b200 as bnb4
 import oracle
-from bit_blockwise_weight_b200 import synthetic
+import synthetic
 
 from gpu_util import to_host
 

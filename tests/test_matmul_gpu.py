@@ -9,7 +9,7 @@ import torch
 
 import bit_blockwise_weight_b200 as bnb4
 import oracle
-from bit_blockwise_weight_b200 import synthetic
+import synthetic
 
 from gpu_util import MATMUL_TOL, as_f64, rel_l2, to_dev, to_host
 

@@ -16,7 +16,7 @@ import torch
 
 import oracle
 from oracle import bruteforce as bf
-from bit_blockwise_weight_b200 import synthetic
+import synthetic
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 

@@ -20,7 +20,7 @@ import pytest
 
 import oracle
 from oracle import bruteforce as bf
-from bit_blockwise_weight_b200 import synthetic
+import synthetic
 
 
 def _to_fracs(arr, dtype):

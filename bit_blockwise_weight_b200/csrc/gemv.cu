@@ -7,25 +7,29 @@
 // turns every weight into an fp32 FMA issues more instructions than HBM lets
 // it retire, so the multiply-adds go to the tensor cores (mma.sync.m16n8k16,
 // fp32 accumulation) and decoding is one byte-permute plus one conflict-free
-// shared load per two weights.
+// shared load per two weights.  Every lane loads 16 contiguous bytes of the
+// weight stream per instruction (narrower loads leave B200's HBM well short
+// of its bandwidth at these sizes).
 //
-// Packing the tensor-core tile.  One MMA multiplies a 16 x 16 A tile by a
-// 16 x 8 B tile.  A row m of A holds 16 weights of row rho(m) of a row pair
-// and item iota(m) of a 512-weight segment (an item is 64 consecutive weights
-// of one row, so it lies in one quantization block):
-//     m = g      (g = 0..7):  rho = g & 1, iota = g >> 1       (items 0..3)
-//     m = g + 8:              rho = g & 1, iota = 4 + (g >> 1)  (items 4..7)
-// and column n of B holds the matching 16 values of x of item n.  Entry
-// C[m, iota(m)] is then a partial dot product of one row over one item: the
-// other 7 columns of each row are never read.  Four MMAs cover the 64 weights
-// of every item, so one unit (a row pair x a segment = 1024 weights) is four
-// MMAs whose 16 useful sums are each scaled by their block's absmax in fp32.
-//
-// K order inside an item: lane (g, t) feeds, in MMA s, packed bytes 2s and
-// 2s + 1 of its 8 bytes [8t, 8t + 8) of the item, so k-slot 2t + e holds
-// weight 16t + 4s + e and k-slot 2t + 8 + e holds 16t + 4s + 2 + e; the B
-// fragment takes x at the same positions.  The reduction over k is a plain
-// sum, so the order is free.
+// Units.  A unit is a quad of rows x a segment of 512 weights (8 items of 64
+// weights; an item lies in one quantization block).  Row pair of items
+// (2p, 2p + 1) of one row is a 64-byte "item pair".  One MMA multiplies a
+// 16 x 16 A tile by a 16 x 8 B tile; eight MMAs cover a unit:
+//   A row m = g (g = 0..7):  row g & 3 of the quad, item pair g >> 2      (pairs 0, 1)
+//   A row m = g + 8:         row g & 3 of the quad, item pair 2 + (g >> 2) (pairs 2, 3)
+// Lane (g, t) holds bytes [16t, 16t + 16) of its two item pairs (two 16-byte
+// loads; a warp's load covers 4 rows x 128 contiguous bytes) and feeds, in
+// MMA s, bytes 2s and 2s + 1 of each: k-slot 2t + e holds weight 4s + e and
+// k-slot 2t + 8 + e holds weight 4s + 2 + e of the lane's 32 weights, which
+// lie in item 2P + (t >> 1) at item offset 32 (t & 1).  Column n of B is item
+// n of the segment: a lane's B slots hold x where its A bytes belong to item n
+// ((t >> 1) == (n & 1)) and zeros elsewhere, so C[m, n] for n in {2P(m),
+// 2P(m) + 1} is the dot product of one row over one item; the other 6
+// columns of each row are never read.  Lane (g, t) holds C[g, 2t..2t+1] and
+// C[g + 8, 2t..2t+1]: it is the lane with the two useful sums of A row g
+// when t == g >> 2, and of A row g + 8 when t == 2 + (g >> 2).  Each sum is
+// scaled by its block's absmax in fp32.  The reduction over k is a plain
+// sum, so the order of the k-slots is free.
 //
 // Decoding: a byte holds two codes (first element in the high nibble).  A
 // 256-entry table maps it to the two codes as a bf16x2 / f16x2 word (lower k
@@ -38,17 +42,21 @@
 // dequantized value.
 //
 // Work split: CTA c owns rows [N c / G, N (c+1) / G) (balanced to one row) and
-// all of K.  Its work is a list of groups (a block of 4 row pairs x one
-// segment), pair-block major; warp w takes a contiguous, balanced range of
-// groups.  Packed weights and absmax go from global memory straight into
-// registers (8-byte loads, full 32-byte sectors), two groups ahead of the
-// MMAs, so no shared-memory bandwidth is spent on staging them; x is staged
-// once per CTA in shared memory (swizzled: the eight items a warp reads at
-// once land in distinct banks).  A lane accumulates its useful sums per row
-// pair in fp32 across segments; when a warp leaves a pair block the sums are
-// reduced across lanes and stored to shared memory, and pair blocks that two
-// warps share are added in warp order at the end, so the result is the same
-// bits on every run.  No global scratch.
+// all of K.  Its work is a list of groups (a quad of rows x kSpan consecutive
+// segments, so each row's bytes are asked for in runs of kSpan x 256 bytes:
+// HBM serves long runs of few rows far better than short runs of many),
+// quad major; warp w takes a contiguous, balanced range of groups.  Packed
+// weights and absmax go from global memory straight into registers, one
+// group ahead of the MMAs; x is staged once per CTA in shared memory (the
+// 16-byte pieces of odd items rotated by two places), beside a zeroed line
+// from which the lanes whose B slots must be zero read, each at a bank its
+// partner lane does not use, so a warp's 16-byte reads never conflict and
+// need no masking.  x sits below the table's 64 KB boundary when it fits
+// there, which leaves half of the SM's L1 to the loads in flight.  A lane
+// accumulates its useful sums of a quad in fp32 across segments; when a warp
+// leaves a quad the sums are reduced across lanes and stored to shared
+// memory, and quads that two warps share are added in warp order at the end,
+// so the result is the same bits on every run.  No global scratch.
 //
 // Double-quantized absmax ("mps-bitsandbytes 0.4.7", Functional API, Double
 // Quantization): with DQ the absmax array arrives as 8-bit codes plus one
@@ -67,15 +75,32 @@ __device__ unsigned int g_gemv_layout_errors = 0;  // launches that found their 
 
 namespace {
 
-constexpr int kWarps = 16;
+// Tunables (measured on B200: 16 warps, groups of 2 segments, two units'
+// MMA chains interleaved; longer groups need more registers than 512
+// threads leave and spill)
+#ifndef BNB4_GEMV_WARPS
+#define BNB4_GEMV_WARPS 16
+#endif
+#ifndef BNB4_GEMV_SPAN
+#define BNB4_GEMV_SPAN 2
+#endif
+constexpr int kWarps = BNB4_GEMV_WARPS;
 constexpr int kThreads = kWarps * 32;
-constexpr int kPairs = 4;                 // row pairs per pair block (8 rows)
+constexpr int kSpan = BNB4_GEMV_SPAN;     // segments per group
+#ifndef BNB4_GEMV_ILV
+#define BNB4_GEMV_ILV 2
+#endif
+constexpr int kIlv = BNB4_GEMV_ILV;       // units whose MMA chains are interleaved
+static_assert(kSpan % kIlv == 0, "a group's units are computed kIlv at a time");
 constexpr int kItems = 8;                 // items (64 weights) per segment
 constexpr int kSegK = kItems * 64;        // 512 weights per row per segment
 constexpr int kMaxRows = 1024;            // rows per CTA
 constexpr int kMaxK = 32768;
 constexpr uint32_t kPage = 65536;         // table alignment and size (256 entries x 256 B)
-constexpr uint32_t kPrefix = kMaxRows * 4 + kWarps * 2 * 8 * 4;  // row sums + warp partials
+constexpr uint32_t kPrefix = kMaxRows * 4 + kWarps * 2 * 4 * 4;  // row sums + warp partials
+constexpr uint32_t kZero = 256;           // zeroed bytes read by the masked B lanes
+// 16-byte pieces of x per thread at the largest K (rounded up to whole groups)
+constexpr int kXPieces = ((kMaxK / kSegK + kSpan - 1) / kSpan * kSpan * kSegK / 8 + kThreads - 1) / kThreads;
 
 // shared loads / stores by 32-bit shared-window address
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
@@ -101,52 +126,46 @@ __device__ __forceinline__ float lds32f(uint32_t a) {
     return v;
 }
 
-// 8 bytes of the weight stream (read once: no L1 allocation); zeros when !ok
-__device__ __forceinline__ uint2 ldg_w8(const uint8_t *p, bool ok) {
-    uint2 v;
-    asm volatile(
-        "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\tmov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\t"
-        "@q ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];\n\t}"
-        : "=r"(v.x), "=r"(v.y)
-        : "l"(p), "r"((int)ok));
+// 16 bytes of the weight stream, absmax words and 8-bit codes: read once,
+// no L1 allocation
+__device__ __forceinline__ uint4 ldg_w16(const uint8_t *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
     return v;
 }
-__device__ __forceinline__ float ldg_f32(const float *p, bool ok) {
+__device__ __forceinline__ float ldg_f32(const float *p) {
     float v;
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\tmov.b32 %0, 0;\n\t"
-                 "@q ld.global.nc.L1::no_allocate.f32 %0, [%1];\n\t}"
-                 : "=f"(v)
-                 : "l"(p), "r"((int)ok));
+    asm volatile("ld.global.nc.L1::no_allocate.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
 }
-__device__ __forceinline__ uint32_t ldg_u8(const uint8_t *p, bool ok) {
+__device__ __forceinline__ uint32_t ldg_u8(const uint8_t *p) {
     uint32_t v;
-    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\tmov.b32 %0, 0;\n\t"
-                 "@q ld.global.nc.L1::no_allocate.u8 %0, [%1];\n\t}"
-                 : "=r"(v)
-                 : "l"(p), "r"((int)ok));
+    asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=r"(v) : "l"(p));
     return v;
 }
 
+// c += A B (run) or c = A B (first: the accumulator input is one zero register)
+#define BNB4_MMA(TY)                                                                                            \
+    __device__ static __forceinline__ void run(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,          \
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {                       \
+        asm("mma.sync.aligned.m16n8k16.row.col.f32." TY "." TY ".f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, " \
+            "{%0,%1,%2,%3};"                                                                                 \
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])                                                 \
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));                                         \
+    }                                                                                                         \
+    __device__ static __forceinline__ void first(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,        \
+                                                 uint32_t a3, uint32_t b0, uint32_t b1) {                     \
+        asm("mma.sync.aligned.m16n8k16.row.col.f32." TY "." TY ".f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, " \
+            "{%10,%10,%10,%10};"                                                                             \
+            : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])                                                 \
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));                              \
+    }
 template <typename D> struct Mma;
-template <> struct Mma<BF16> {
-    __device__ static __forceinline__ void run(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
-};
-template <> struct Mma<F16> {
-    __device__ static __forceinline__ void run(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-        asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-            "{%0,%1,%2,%3};"
-            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-    }
-};
+template <> struct Mma<BF16> { BNB4_MMA("bf16") };
+template <> struct Mma<F16> { BNB4_MMA("f16") };
+#undef BNB4_MMA
 
 // table lookup of byte k (0..3) of w: prmt puts the lane's bank offset in
 // byte 0, the packed byte in byte 1 and the table page in bytes 2..3 of the
@@ -156,13 +175,17 @@ __device__ __forceinline__ uint32_t lut(uint32_t w, uint32_t L) {
     return lds32(prmt(w, L, 0x7604u | (k << 4)));
 }
 
-// one unit's loads: 8 packed bytes of item iota(g) and of item iota(g + 8),
-// and, on the lane that scales a sum, its block's absmax (or 8-bit code and
-// group scale)
+__device__ __forceinline__ uint32_t word(const uint4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// one unit's loads (a unit is a quad x one segment): the lane's 16 bytes of
+// its two item pairs and, on the lane that scales sums, the absmax (or 8-bit
+// codes and group scales) of its two items
 struct Unit {
-    uint2 wa, wb;
-    float am;
-    uint32_t code;
+    uint4 wa, wb;
+    float am0, am1;
+    uint32_t code0, code1;
 };
 
 }  // namespace
@@ -177,16 +200,20 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t base0 = (uint32_t)__cvta_generic_to_shared(smem);
     const uint32_t rowsum_a = base0;                         // float [kMaxRows]
-    const uint32_t part_a = base0 + kMaxRows * 4;            // float [kWarps][2][8]
-    const uint32_t lut_a = (base0 + kPrefix + kPage - 1) & ~(kPage - 1);
-    const uint32_t xs_a = lut_a + kPage;
+    const uint32_t part_a = base0 + kMaxRows * 4;            // float [kWarps][2][4]
+    const uint32_t zero_a = base0 + kPrefix;                 // kZero bytes of zeros
+    const uint32_t lut_a = (zero_a + kZero + kPage - 1) & ~(kPage - 1);
 
     const int nitems = K >> 6;
-    const int S = (nitems + kItems - 1) / kItems;
+    const int S = (nitems + kItems - 1) / kItems;            // segments per row
+    const int SS = (S + kSpan - 1) / kSpan;                  // groups per quad
+    const uint32_t xbytes = (uint32_t)SS * kSpan * kSegK * 2;
+    // item i of x at xs_a + 128 i: below the table if it fits, else above it
+    const uint32_t xs_a = zero_a + kZero + xbytes <= lut_a ? zero_a + kZero : lut_a + kPage;
     {
         uint32_t dyn;
         asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
-        if (xs_a + (uint32_t)S * kSegK * 2 > base0 + dyn) {
+        if (xs_a + xbytes > base0 + dyn || lut_a + kPage > base0 + dyn) {
             // the shared-memory plan does not fit the launch: report, write nothing
             if (threadIdx.x == 0) atomicAdd(&g_gemv_layout_errors, 1u);
             return;
@@ -198,153 +225,247 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
     const int r0 = (int)(((int64_t)N * blockIdx.x) / G);
     const int r1 = (int)(((int64_t)N * (blockIdx.x + 1)) / G);
     const int R = r1 - r0;
-    const int NP = (R + 1) >> 1;
-    const int NPB = (NP + kPairs - 1) / kPairs;
-    const int GU = NPB * S;                                  // groups of this CTA
+    const int NQ = (R + 3) >> 2;                             // quads
+    const int GU = NQ * SS;                                  // groups of this CTA
     const int g_lo = (int)(((int64_t)GU * warp) / kWarps);
     const int g_hi = (int)(((int64_t)GU * (warp + 1)) / kWarps);
 
     const int g8 = lane >> 2, t4 = lane & 3;
-    const int rho = g8 & 1, itA = g8 >> 1;
-    // the lane's useful accumulator entry (at most one per lane)
+    const int rq = g8 & 3;                                   // row within the quad
+    const int pA = g8 >> 2, pB = 2 + (g8 >> 2);              // the lane's item pairs
+    // the lane's useful sums (two, of one A row), if any
     const bool hiC = t4 >= 2;
     const bool useful = t4 == (g8 >> 2) || t4 == 2 + (g8 >> 2);
-    const bool oddC = (itA & 1) != 0;
-    const int it_u = hiC ? itA + 4 : itA;
+    const int it_u = 2 * (hiC ? pB : pA);                    // first of its two items
     const int64_t row_bytes = K >> 1;
     const int nblk = K >> log2B;
     const int bsh = log2B - 6;                               // item -> block
+    const uint8_t *Wt = W + (int64_t)r0 * row_bytes + 64 * pA + 16 * t4;
+    const int64_t a0 = (int64_t)r0 * nblk;
 
-    auto load = [&](int g, Unit (&u)[kPairs]) {
-        const int pb = g / S, j = g - pb * S;
-        const int iA = j * kItems + itA, iB = iA + 4, iu = j * kItems + it_u;
+    // Loads of group (q, ss).  Rows past the CTA's last row and items past K
+    // are clamped to the last ones: they read real data, whose sums are never
+    // stored (rows) or meet zeros of x (items), so no load is predicated.
+    auto load = [&](int q, int ss, Unit (&u)[kSpan]) {
+        const int rl = min(4 * q + rq, R - 1);
+        const int64_t br = a0 + (int64_t)rl * nblk;
+        const int j0 = ss * kSpan;
+        if (!DQ && bsh == 0 && (ss + 1) * kSpan * kItems <= nitems) {
+            // the common case (blocks of 64, every item of the group in K): one
+            // base address per group, the units at immediate offsets
+            const uint8_t *wg = Wt + (int64_t)rl * row_bytes + 256 * j0;
+            const float *ag = static_cast<const float *>(absmax) + br + kItems * j0 + it_u;
 #pragma unroll
-        for (int pp = 0; pp < kPairs; ++pp) {
-            const int rl = 2 * (pb * kPairs + pp) + rho;     // row within the CTA
-            const bool rok = rl < R && g < g_hi;
-            const int row = r0 + rl;
-            const uint8_t *wr = W + (int64_t)row * row_bytes + 8 * t4;
-            u[pp].wa = ldg_w8(wr + iA * 32, rok && iA < nitems);
-            u[pp].wb = ldg_w8(wr + iB * 32, rok && iB < nitems);
-            const bool aok = rok && useful && iu < nitems;
-            const int64_t bi = (int64_t)row * nblk + (iu >> bsh);
-            if constexpr (DQ) {
-                u[pp].code = ldg_u8(static_cast<const uint8_t *>(absmax) + (aok ? bi : 0), aok);
-                u[pp].am = ldg_f32(scales + (aok ? (bi >> log2G) : 0), aok);
+            for (int sp = 0; sp < kSpan; ++sp) {
+                u[sp].wa = ldg_w16(wg + 256 * sp);
+                u[sp].wb = ldg_w16(wg + 256 * sp + 128);
+                u[sp].am0 = ldg_f32(ag + kItems * sp);
+                u[sp].am1 = ldg_f32(ag + kItems * sp + 1);
+                u[sp].code0 = u[sp].code1 = 0;
+            }
+            return;
+        }
+        const uint8_t *wr = Wt + (int64_t)rl * row_bytes;
+        const bool whole = (ss + 1) * kSpan * kItems <= nitems;  // every item of the group is in K
+#pragma unroll
+        for (int sp = 0; sp < kSpan; ++sp) {
+            const int j = j0 + sp;
+            if (whole) {
+                u[sp].wa = ldg_w16(wr + 256 * j);
+                u[sp].wb = ldg_w16(wr + 256 * j + 128);
             } else {
-                u[pp].am = ldg_f32(static_cast<const float *>(absmax) + (aok ? bi : 0), aok);
-                u[pp].code = 0;
+                // byte offsets of the lane's chunks with their items clamped to K
+                const int iA = min(j * kItems + 2 * pA + (t4 >> 1), nitems - 1);
+                const int iB = min(j * kItems + 2 * pB + (t4 >> 1), nitems - 1);
+                const uint8_t *wc = wr - 64 * pA - 16 * t4 + 16 * (t4 & 1);
+                u[sp].wa = ldg_w16(wc + 32 * iA);
+                u[sp].wb = ldg_w16(wc + 32 * iB);
+            }
+            const int b0 = min(j * kItems + it_u, nitems - 1) >> bsh;
+            const int b1 = min(j * kItems + it_u + 1, nitems - 1) >> bsh;
+            if constexpr (DQ) {
+                const uint8_t *q8 = static_cast<const uint8_t *>(absmax);
+                u[sp].code0 = ldg_u8(q8 + br + b0);
+                u[sp].code1 = ldg_u8(q8 + br + b1);
+                u[sp].am0 = ldg_f32(scales + ((br + b0) >> log2G));
+                u[sp].am1 = ldg_f32(scales + ((br + b1) >> log2G));
+            } else {
+                const float *af = static_cast<const float *>(absmax);
+                u[sp].am0 = ldg_f32(af + br + b0);
+                u[sp].am1 = ldg_f32(af + br + b1);
+                u[sp].code0 = u[sp].code1 = 0;
             }
         }
     };
 
-    Unit ua[kPairs], ub[kPairs];
-    // the first two groups' loads leave before the table and x are staged
-    load(g_lo, ua);
-    load(g_lo + 1, ub);
+    // this warp's groups, visited in order: (quad, span) advance without divisions
+    const int ng = g_hi - g_lo;
+    int cq = 0, css = 0;
+    if (ng > 0) {
+        cq = g_lo / SS;
+        css = g_lo - cq * SS;
+    }
+    const int q_first = ng > 0 ? cq : -1;
+    const int q_last = ng > 0 ? (g_hi - 1) / SS : -1;
+
+    Unit ua[kSpan], ub[kSpan];
+    // the first group's loads leave before the table and x are staged
+    if (ng > 0) load(cq, css, ua);
     {
         // table: entry v (codes of nibbles v >> 4, v & 15) copied to words 64 v + l, l < 32
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2048 / kThreads; ++i) {
             const int idx = tid + i * kThreads;              // 2048 16-byte pieces
             const int v = idx >> 3, q = idx & 7;
             const uint32_t e = Dt<D>::pack2(tab.v[v >> 4], tab.v[v & 15]);
             sts128(lut_a + v * 256 + q * 16, make_uint4(e, e, e, e));
         }
-        // x: 16-byte piece q of item i at position (q + (i & 1)) & 7; zeros past K
+        if (tid < kZero / 16) sts128(zero_a + 16 * tid, make_uint4(0, 0, 0, 0));
+        // x: 16-byte piece q of item i at position (q + 2 (i & 1)) & 7 of the
+        // item's 128 bytes; zeros past K.  All of a thread's loads leave before
+        // any store, so staging costs one round trip.
         const uint4 *x4 = reinterpret_cast<const uint4 *>(x);
-        const int npieces = S * kSegK / 8;
-        for (int c = tid; c < npieces; c += kThreads) {
-            const uint4 v = 8 * c < K ? __ldg(x4 + c) : make_uint4(0, 0, 0, 0);
-            const int i = c >> 3, q = c & 7;
-            sts128(xs_a + i * 128 + (((q + (i & 1)) & 7) << 4), v);
+        const int npieces = SS * kSpan * kSegK / 8;
+        uint4 xv[kXPieces];
+#pragma unroll
+        for (int i = 0; i < kXPieces; ++i) {
+            const int c = tid + i * kThreads;
+            xv[i] = 8 * c < K ? __ldg(x4 + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kXPieces; ++i) {
+            const int c = tid + i * kThreads, it = c >> 3;
+            if (c < npieces) sts128(xs_a + it * 128 + ((((c & 7) + 2 * (it & 1)) & 7) << 4), xv[i]);
         }
     }
     __syncthreads();
 
     const uint32_t L = lut_a | (4u * lane);
-    const int pb_first = g_lo < g_hi ? g_lo / S : -1;
-    const int pb_last = g_lo < g_hi ? (g_hi - 1) / S : -1;
-    float acc[kPairs] = {0.f, 0.f, 0.f, 0.f};
-
-    // reduce the lanes' sums of pair block pb and store its 8 row sums
-    auto flush = [&](int pb) {
-        const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0;
-        // over lane bit 4: keep pairs (0, 1) or (2, 3), send the other two
-        float k0 = b4 ? acc[2] : acc[0], k1 = b4 ? acc[3] : acc[1];
-        const float s0 = b4 ? acc[0] : acc[2], s1 = b4 ? acc[1] : acc[3];
-        k0 += __shfl_xor_sync(FULL, s0, 16);
-        k1 += __shfl_xor_sync(FULL, s1, 16);
-        // over lane bit 3: keep one of the two
-        float q = b3 ? k1 : k0;
-        q += __shfl_xor_sync(FULL, b3 ? k0 : k1, 8);
-        q += __shfl_xor_sync(FULL, q, 1);
-        q += __shfl_xor_sync(FULL, q, 2);
-        // lanes 4 i hold pair 2 b4 + b3, row rho = bit 2
-        if ((lane & 3) == 0) {
-            const int k = 2 * (2 * (int)b4 + (int)b3) + ((lane >> 2) & 1);  // row within the block
-            if (pb == pb_first)
-                sts32f(part_a + (warp * 16 + k) * 4, q);
-            else if (pb == pb_last)
-                sts32f(part_a + (warp * 16 + 8 + k) * 4, q);
-            else if (8 * pb + k < R)
-                sts32f(rowsum_a + (8 * pb + k) * 4, q);
-        }
+    // B: x of item g8 at the lane's half (t4 & 1) of it where the lane's bytes
+    // lie in that item ((t4 >> 1) == (g8 & 1)); zeros elsewhere, read from the
+    // zeroed line one piece past the partner lane's bank group
+    const bool bmask = (t4 >> 1) == (g8 & 1);
+    const uint32_t xbase = bmask ? xs_a + g8 * 128 : zero_a;
+    const uint32_t xstride = bmask ? kItems * 128 : 0;
+    uint32_t xo[4];
 #pragma unroll
-        for (int pp = 0; pp < kPairs; ++pp) acc[pp] = 0.f;
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t pos = (4 * (t4 & 1) + q + 2 * (g8 & 1)) & 7;
+        xo[q] = (bmask ? pos : (pos + 1) & 7) << 4;
+    }
+    float acc = 0.f;
+
+    // reduce the lanes' sums of quad q and store its 4 row sums
+    auto flush = [&](int q) {
+        float v = acc;
+        v += __shfl_xor_sync(FULL, v, 16);
+        v += __shfl_xor_sync(FULL, v, 1);
+        v += __shfl_xor_sync(FULL, v, 2);
+        if ((lane & 19) == 0) {                              // lanes 0, 4, 8, 12: rows 0..3
+            const int k = (lane >> 2) & 3;
+            if (q == q_first)
+                sts32f(part_a + (warp * 8 + k) * 4, v);
+            else if (q == q_last)
+                sts32f(part_a + (warp * 8 + 4 + k) * 4, v);
+            else if (4 * q + k < R)
+                sts32f(rowsum_a + (4 * q + k) * 4, v);
+        }
+        acc = 0.f;
     };
 
-    auto compute = [&](int g, const Unit (&u)[kPairs]) {
-        const int pb = g / S, j = g - pb * S;
-        // x of item 8 j + g8 at this lane's 16 positions [16 t, 16 t + 16)
-        const uint32_t xi = xs_a + (j * kItems + g8) * 128;
-        const uint4 x0 = lds128(xi + (((2 * t4 + (g8 & 1)) & 7) << 4));
-        const uint4 x1 = lds128(xi + (((2 * t4 + 1 + (g8 & 1)) & 7) << 4));
+    // kIlv units' MMA chains at a time are interleaved; rows past the CTA's
+    // rows are computed on clamped data and never stored
+    auto compute = [&](int ss, const Unit (&u)[kSpan]) {
 #pragma unroll
-        for (int pp = 0; pp < kPairs; ++pp) {
-            if (2 * (pb * kPairs + pp) < R) {                 // warp-uniform
-                float c[4] = {0.f, 0.f, 0.f, 0.f};
-                const uint32_t wa0 = u[pp].wa.x, wa1 = u[pp].wa.y, wb0 = u[pp].wb.x, wb1 = u[pp].wb.y;
-                Mma<D>::run(c, lut<0>(wa0, L), lut<0>(wb0, L), lut<1>(wa0, L), lut<1>(wb0, L), x0.x, x0.y);
-                Mma<D>::run(c, lut<2>(wa0, L), lut<2>(wb0, L), lut<3>(wa0, L), lut<3>(wb0, L), x0.z, x0.w);
-                Mma<D>::run(c, lut<0>(wa1, L), lut<0>(wb1, L), lut<1>(wa1, L), lut<1>(wb1, L), x1.x, x1.y);
-                Mma<D>::run(c, lut<2>(wa1, L), lut<2>(wb1, L), lut<3>(wa1, L), lut<3>(wb1, L), x1.z, x1.w);
-                float v = hiC ? (oddC ? c[3] : c[2]) : (oddC ? c[1] : c[0]);
-                v = useful ? v : 0.f;
-                float am = u[pp].am;
-                if constexpr (DQ) {
-                    const float cf = __uint_as_float(0x4b000000u | u[pp].code) - 8388608.0f;
-                    am = useful ? __fmul_rn(cf, div255_rn(am)) : 0.f;
+        for (int h = 0; h < kSpan; h += kIlv) {
+            float c[kIlv][4];
+            uint32_t xr[kIlv][16];
+#pragma unroll
+            for (int e = 0; e < kIlv; ++e) {
+                const uint32_t xa = xbase + (uint32_t)(ss * kSpan + h + e) * xstride;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 v = lds128(xa + xo[q]);
+                    xr[e][4 * q] = v.x;
+                    xr[e][4 * q + 1] = v.y;
+                    xr[e][4 * q + 2] = v.z;
+                    xr[e][4 * q + 3] = v.w;
                 }
-                acc[pp] = __fmaf_rn(v, am, acc[pp]);
+            }
+#pragma unroll
+            for (int st = 0; st < 8; ++st) {
+#pragma unroll
+                for (int e = 0; e < kIlv; ++e) {
+                    const Unit &un = u[h + e];
+                    const uint32_t wa = word(un.wa, st >> 1), wb = word(un.wb, st >> 1);
+                    if (st == 0)
+                        Mma<D>::first(c[e], lut<0>(wa, L), lut<0>(wb, L), lut<1>(wa, L), lut<1>(wb, L), xr[e][0],
+                                      xr[e][1]);
+                    else if (st & 1)
+                        Mma<D>::run(c[e], lut<2>(wa, L), lut<2>(wb, L), lut<3>(wa, L), lut<3>(wb, L),
+                                    xr[e][2 * st], xr[e][2 * st + 1]);
+                    else
+                        Mma<D>::run(c[e], lut<0>(wa, L), lut<0>(wb, L), lut<1>(wa, L), lut<1>(wb, L),
+                                    xr[e][2 * st], xr[e][2 * st + 1]);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < kIlv; ++e) {
+                const Unit &un = u[h + e];
+                float v0 = hiC ? c[e][2] : c[e][0];
+                float v1 = hiC ? c[e][3] : c[e][1];
+                v0 = useful ? v0 : 0.f;
+                v1 = useful ? v1 : 0.f;
+                float am0 = un.am0, am1 = un.am1;
+                if constexpr (DQ) {
+                    am0 = __fmul_rn(__uint_as_float(0x4b000000u | un.code0) - 8388608.0f, div255_rn(am0));
+                    am1 = __fmul_rn(__uint_as_float(0x4b000000u | un.code1) - 8388608.0f, div255_rn(am1));
+                }
+                acc = __fmaf_rn(v0, am0, acc);
+                acc = __fmaf_rn(v1, am1, acc);
             }
         }
-        if (g + 1 == g_hi || (g + 1) / S != pb) flush(pb);
     };
 
-    for (int g = g_lo; g < g_hi; g += 2) {
-        compute(g, ua);
-        load(g + 2, ua);
-        if (g + 1 < g_hi) {
-            compute(g + 1, ub);
-            load(g + 3, ub);
+    auto next = [&](int &q, int &ss) {
+        if (++ss == SS) {
+            ss = 0;
+            ++q;
+        }
+    };
+    // ua holds group i, ub group i + 1 (loaded while group i is computed)
+    for (int i = 0; i < ng; i += 2) {
+        int nq = cq, nss = css;
+        next(nq, nss);
+        if (i + 1 < ng) load(nq, nss, ub);
+        compute(css, ua);
+        if (i + 1 == ng || nq != cq) flush(cq);
+        if (i + 1 < ng) {
+            cq = nq;
+            css = nss;
+            next(nq, nss);
+            if (i + 2 < ng) load(nq, nss, ua);
+            compute(css, ub);
+            if (i + 2 == ng || nq != cq) flush(cq);
+            cq = nq;
+            css = nss;
         }
     }
     __syncthreads();
 
     for (int r = tid; r < R; r += kThreads) {
-        // the warps whose group ranges meet this row's pair block (groups
-        // [ul, uh)), in order.  A warp starting inside the block left it in
-        // slot 0, one ending inside it in slot 1; otherwise the block is the
-        // warp's alone and went to the row sums.
-        const int pb = r >> 3, k = r & 7, ul = pb * S, uh = ul + S;
+        // the warps whose group ranges meet this row's quad (groups [ul, uh)),
+        // in order.  A warp starting inside the quad left it in slot 0, one
+        // ending inside it in slot 1; otherwise the quad is the warp's alone
+        // and went to the row sums.
+        const int q = r >> 2, k = r & 3, ul = q * SS, uh = ul + SS;
         const int w0 = (kWarps * (ul + 1) + GU - 1) / GU - 1, w1 = (kWarps * uh + GU - 1) / GU - 1;
         float v = 0.f;
         for (int w = w0; w <= w1; ++w) {
             const int lo = (int)(((int64_t)GU * w) / kWarps), hi = (int)(((int64_t)GU * (w + 1)) / kWarps);
             if (lo >= hi) continue;
-            v += lo >= ul ? lds32f(part_a + (w * 16 + k) * 4)
-                 : hi - 1 < uh ? lds32f(part_a + (w * 16 + 8 + k) * 4)
+            v += lo >= ul ? lds32f(part_a + (w * 8 + k) * 4)
+                 : hi - 1 < uh ? lds32f(part_a + (w * 8 + 4 + k) * 4)
                                : lds32f(rowsum_a + r * 4);
         }
         if (bias) v += Dt<D>::to_f32(bias[r0 + r]);
@@ -354,13 +475,18 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
 
 namespace {
 
-// shared memory the kernel asks for: the prefix, padding up to the next 64 KB
-// boundary of the shared window (the dynamic region starts right after the
-// device's reserved shared memory), the table and x
+// shared memory the kernel asks for: the prefix, the zeroed line, x when it
+// fits below the next 64 KB boundary of the shared window (the dynamic region
+// starts right after the device's reserved shared memory), the table, and x
+// above it otherwise
 size_t smem_bytes(int K, int reserved) {
     const size_t S = ((size_t)(K >> 6) + kItems - 1) / kItems;
-    const size_t lut = ((size_t)reserved + kPrefix + kPage - 1) / kPage * kPage;
-    return lut - (size_t)reserved + kPage + S * kSegK * 2;
+    const size_t SS = (S + kSpan - 1) / kSpan;
+    const size_t xbytes = SS * kSpan * kSegK * 2;
+    const size_t zero = (size_t)reserved + kPrefix;
+    const size_t lut = (zero + kZero + kPage - 1) / kPage * kPage;
+    const size_t end = zero + kZero + xbytes <= lut ? lut + kPage : lut + kPage + xbytes;
+    return end - (size_t)reserved;
 }
 
 template <typename D, bool DQ>

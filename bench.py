@@ -181,19 +181,23 @@ def job_rate(units_per_rank_step: float, steps: int, world: int, ms: float) -> f
     return units_per_rank_step * steps * world / (ms / 1e3)
 
 
-def roofline_and_parts(ops, per_op_ms, hbm, tc_sust, peak_kind, traffic=None):
+def roofline_and_parts(ops, per_op_ms, hbm, tc_burst, tc_sust, peak_kind, traffic=None):
     """The roofline object for the op with the largest time share (HBM GB/s, or
     TFLOP/s for the tensor-core matmuls) and the per-op breakdown.
-    ops: (name, algorithmic bytes, flops) per launch; per_op_ms: mean durations."""
+    ops: (name, algorithmic bytes, flops) per launch; per_op_ms: mean durations.
+    A tensor-core op is judged against the burst bf16 peak (its launches are tens
+    of microseconds inside a sub-millisecond step, not a seconds-long loop under
+    the power cap); the fraction of the sustained peak is reported beside it."""
     traffic = traffic or profiled_traffic
     di = max(range(len(per_op_ms)), key=lambda i: per_op_ms[i])
     name, nbytes, nflops = ops[di]
     if nflops and "_M512_" in name:
         achieved = nflops / (per_op_ms[di] / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_sust,
-                "unit": "TFLOP/s", "frac": round(achieved / tc_sust, 4),
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tc_burst,
+                "unit": "TFLOP/s", "frac": round(achieved / tc_burst, 4),
+                "frac_of_sustained": round(achieved / tc_sust, 4),
                 "traffic": traffic(name), "kernel": name,
-                "peak_kind": f"{peak_kind} sustained bf16"}
+                "peak_kind": f"{peak_kind} burst bf16 (sustained {tc_sust})"}
     else:
         achieved = nbytes / (per_op_ms[di] / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
@@ -207,9 +211,146 @@ def roofline_and_parts(ops, per_op_ms, hbm, tc_sust, peak_kind, traffic=None):
              "share": round(t / total, 4)}
         if "_M512_" in nm:
             e["TFLOP/s"] = round(nf / (t / 1e3) / 1e12, 1)
-            e["tensor_frac"] = round(nf / (t / 1e3) / 1e12 / tc_sust, 4)
+            e["tensor_frac"] = round(nf / (t / 1e3) / 1e12 / tc_burst, 4)
+            e["tensor_frac_of_sustained"] = round(nf / (t / 1e3) / 1e12 / tc_sust, 4)
         parts[nm] = e
     return roof, parts
+
+
+def graph_per_launch(dev, fns, reps=5):
+    """Mean device time of one launch, in microseconds: the launches (zero-argument
+    callables) captured back to back in one CUDA graph, replayed `reps` times
+    between two events on the stream the replays run on, after one untimed
+    replay.  The
+    callers rotate inputs whose total size exceeds L2, so every launch reads cold
+    data."""
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    for f in fns[:2]:
+        f()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for f in fns:
+            f()
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    # replay() launches on the current stream: the events go there too
+    cur = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cur)
+    for _ in range(reps):
+        g.replay()
+    e1.record(cur)
+    torch.cuda.synchronize(dev)
+    del g
+    return e0.elapsed_time(e1) * 1e3 / (reps * len(fns))
+
+
+def copies_for(nbytes, floor_bytes=640 << 20):
+    """How many rotating copies of an input of `nbytes` keep the working set of
+    one pass above five times L2."""
+    return max(2, -(-floor_bytes // max(nbytes, 1)))
+
+
+def time_configs(dev, hbm, tc_burst, tc_sust):
+    """Every workload configuration of the path, each op timed on its own with
+    graph_per_launch: quantize/dequantize 2^28 (3 dtypes x NF4/FP4 x 7
+    blocksizes), the gemv decode shapes with and without bias (the 4096 x 4096
+    one is the gemv NF4 workload), small-M decode on the 70B shapes (M = 1, 2,
+    4, 8, 16 x NF4/FP4 x bf16/fp16) and prefill M = 512 / 2048 forward and
+    backward."""
+    import bit_blockwise_weight_b200 as b
+    import synthetic
+    d = str(dev)
+    out = {}
+
+    def rec(name, us, nbytes, flops=0):
+        e = {"us": round(us, 2), "bytes": int(nbytes), "GB/s": round(nbytes / (us / 1e6) / 1e9, 1),
+             "hbm_frac": round(nbytes / (us / 1e6) / 1e9 / hbm, 4)}
+        if flops:
+            tf = flops / (us / 1e6) / 1e12
+            e.update({"TFLOP/s": round(tf, 1), "tensor_frac": round(tf / tc_burst, 4),
+                      "tensor_frac_of_sustained": round(tf / tc_sust, 4)})
+        out[name] = e
+
+    def qweight(N, K, sigma, seed, qt, copies):
+        w = synthetic.normal((N * K,), seed, sigma, "f32", device=d)
+        p, a = b.quantize_4bit(w, BLOCK, qt)
+        del w
+        return [p] + [p.clone() for _ in range(copies - 1)], [a] + [a.clone() for _ in range(copies - 1)]
+
+    # quantize / dequantize round trip, 2^28 elements (the input is 0.5-1 GB: each
+    # launch reads cold data)
+    n = N_ELEMS
+    packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    for dt, tdt in (("f32", torch.float32), ("f16", torch.float16), ("bf16", torch.bfloat16)):
+        x = synthetic.roundtrip_tensor(n, 0, dt, device=d)
+        y = torch.empty(n, dtype=tdt, device=dev)
+        s = x.element_size()
+        for qt in ("nf4", "fp4"):
+            for B in (64, 128, 256, 512, 1024, 2048, 4096):
+                nb = n * s + n // 2 + 4 * (n // B)
+                a_ = absmax[: n // B]
+                us = graph_per_launch(dev, [lambda: b.quantize_4bit_into(x, packed, a_, B, qt)] * 2, reps=3)
+                rec(f"quantize_4bit_2p28_{dt}_{qt}_B{B}", us, nb)
+                us = graph_per_launch(dev, [lambda: b.dequantize_4bit(packed, a_, n, B, qt, out=y)] * 2, reps=3)
+                rec(f"dequantize_4bit_2p28_{dt}_{qt}_B{B}", us, nb)
+        del x, y
+    del packed, absmax
+
+    # gemv decode shapes (the 4096 x 4096 NF4 one without bias is the gemv NF4 workload)
+    for K, N in GEMV_SHAPES:
+        nbw = wbytes(N, K)
+        C = copies_for(nbw)
+        ps, as_ = qweight(N, K, 0.02, 0, "nf4", C)
+        xv = synthetic.normal((K,), 1, 1.0, "bf16", device=d)
+        bias = synthetic.normal((N,), 2, 1.0, "bf16", device=d)
+        y = torch.empty(N, dtype=torch.bfloat16, device=dev)
+        for with_bias in (False, True):
+            fns = [lambda i=i: b.gemv_4bit(xv, ps[i], as_[i], N, K, bias if with_bias else None, BLOCK, "nf4",
+                                           out=y) for i in range(C)]
+            us = graph_per_launch(dev, fns)
+            rec(f"gemv_4bit_nf4_bf16_{K}x{N}" + ("_bias" if with_bias else ""), us,
+                nbw + 2 * K + 2 * N + (2 * N if with_bias else 0), 2 * N * K)
+        del ps, as_
+
+    # small-M decode, 70B-shaped (133 MB of weight: two rotating copies)
+    for K, N in SMALLM_SHAPES:
+        nbw = wbytes(N, K)
+        for qt in ("nf4", "fp4"):
+            ps, as_ = qweight(N, K, 0.015, 0, qt, 2)
+            for dt, tdt in (("bf16", torch.bfloat16), ("f16", torch.float16)):
+                for M in (1, 2, 4, 8, 16):
+                    X = synthetic.normal((M, K), 1, 1.0, dt, device=d)
+                    Y = torch.empty(M, N, dtype=tdt, device=dev)
+                    fns = [lambda i=i: b.gemm_4bit(X, ps[i], as_[i], N, None, BLOCK, qt, out=Y) for i in range(2)]
+                    us = graph_per_launch(dev, fns)
+                    rec(f"gemm_4bit_M{M}_{qt}_{dt}_{K}x{N}", us, nbw + 2 * M * K + 2 * M * N, 2 * M * N * K)
+            del ps, as_
+
+    # prefill forward and backward
+    M0, K, N = PREFILL
+    ps, as_ = qweight(N, K, 0.02, 0, "nf4", 2)
+    for M in (512, 2048):
+        X = synthetic.normal((M, K), 4000, 1.0, "bf16", device=d)
+        dY = synthetic.normal((M, N), 5000, 1.0, "bf16", device=d)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+        fl = 2 * M * N * K
+        us = graph_per_launch(dev, [lambda i=i: b.gemm_4bit(X, ps[i], as_[i], N, None, BLOCK, "nf4", out=Y)
+                                    for i in range(2)])
+        rec(f"gemm_4bit_M{M}_nf4_bf16_{K}x{N}", us, wbytes(N, K) + 2 * M * K + 2 * M * N, fl)
+        us = graph_per_launch(dev, [lambda i=i: b.gemm_4bit_backward(dY, ps[i], as_[i], K, BLOCK, "nf4", out=dX)
+                                    for i in range(2)])
+        rec(f"gemm_4bit_backward_M{M}_nf4_bf16_{K}x{N}", us, wbytes(N, K) + 2 * M * N + 2 * M * K, fl)
+    del ps, as_
+    out["note"] = ("each op alone: its launches back to back in one CUDA graph over rotating copies of its "
+                   "inputs (the working set of a pass is above 5x L2, so every launch reads cold data); "
+                   "time per launch = replay time / launches")
+    return out
 
 
 # ----------------------------------------------------------------- our arm
@@ -336,8 +477,9 @@ def run_ours(args, rank, world, dev):
     value = job_rate(step_bytes, args.steps, world, ms) / 1e9
 
     # the next rows beyond the step (double-quantized statistics), timed on their own
-    next_rows = time_next_rows(step, dev, args.steps, hbm)
-    next_rows.update(time_8bit_and_embedding(dev, min(args.steps, 10), hbm))
+    next_rows = time_next_rows(step, dev, hbm)
+    next_rows.update(time_8bit_and_embedding(dev, hbm))
+    configs = time_configs(dev, hbm, tc_burst, tc_sust)
 
     # e2e: the same step through the public API from pinned host buffers; the step's
     # inputs go host->device and every output comes back device->host, every step
@@ -345,7 +487,7 @@ def run_ours(args, rank, world, dev):
 
     if rank != 0:
         return None
-    roof, parts = roofline_and_parts(ops, per_op_ms, hbm, tc_sust, peak_kind)
+    roof, parts = roofline_and_parts(ops, per_op_ms, hbm, tc_burst, tc_sust, peak_kind)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
@@ -355,8 +497,10 @@ def run_ours(args, rank, world, dev):
         "timing": "step captured once as a CUDA graph of its launches; K replays between two "
                   "events; per-launch times from a second graph with an event node after each "
                   "launch",
+        "metric_values": metric_values(configs),
         "roofline": roof,
         "parts": parts,
+        "configs_timed": configs,
         "next_rows": next_rows,
         "e2e": e2e,
         "gpu_launches": len(calls) * args.steps,
@@ -368,67 +512,68 @@ def run_ours(args, rank, world, dev):
     return line
 
 
-def time_next_rows(step, dev, steps, hbm):
+def metric_values(configs):
+    """The metric's own numbers, from the per-config timings: gemv_4bit on the
+    gemv NF4 workload (4096 x 4096, no bias, bf16) in GB/s and as a fraction of
+    the measured HBM copy bandwidth, and quantize_4bit of 2^28 elements (NF4,
+    blocksize 64) in GB/s for the three input dtypes."""
+    out = {}
+    g = configs.get("gemv_4bit_nf4_bf16_4096x4096")
+    if g:
+        out["gemv_4bit_nf4_4096x4096"] = {k: g[k] for k in ("us", "GB/s", "hbm_frac")}
+    for dt in ("bf16", "f16", "f32"):
+        q = configs.get(f"quantize_4bit_2p28_{dt}_nf4_B64")
+        if q:
+            out[f"quantize_4bit_2p28_{dt}_nf4_B64"] = {k: q[k] for k in ("us", "GB/s", "hbm_frac")}
+    return out
+
+
+def time_next_rows(step, dev, hbm):
     """Double quantization of absmax and the gemv on 8-bit statistics, outside
-    the step: double_quant / dequant_absmax on the step's absmax (2^22 values,
-    groups of 256), and each gemv shape with fp32 absmax and with its
-    double-quantized absmax, side by side.  L2 is flushed (a 512 MB fill)
-    before every op; one CUDA graph holds flush, event, op, event per op."""
-    b = step.bnb4
+    the step: double_quant / dequant_absmax of 2^22 absmax values (groups of
+    256), and each gemv decode shape (with bias) on fp32 absmax and on its
+    double-quantized absmax, side by side.  Each op timed with
+    graph_per_launch over rotating copies of its inputs."""
+    import bit_blockwise_weight_b200 as b
     G = 256
     n = step.absmax.numel()
-    aq = torch.empty(n, dtype=torch.uint8, device=dev)
-    asc = torch.empty((n + G - 1) // G, dtype=torch.float32, device=dev)
-    back = torch.empty(n, dtype=torch.float32, device=dev)
-    b.double_quant(step.absmax, G, out=(aq, asc))
-    ops = [("double_quant_absmax_4194304", 4 * n + n + 4 * asc.numel(),
-            lambda: b.double_quant(step.absmax, G, out=(aq, asc))),
-           ("dequant_absmax_4194304", n + 4 * asc.numel() + 4 * n,
-            lambda: b.dequant_absmax(aq, asc, G, out=back))]
-    for K, N, p, a, xv, bias, y in step.gemv:
-        q8, s8 = b.double_quant(a, G)
-        nb = N * K // BLOCK
-        ops.append((f"gemv_4bit_{K}x{N}", N * K // 2 + 4 * nb + 2 * K + 4 * N,
-                    lambda K=K, N=N, p=p, a=a, xv=xv, bias=bias, y=y:
-                    b.gemv_4bit(xv, p, a, N, K, bias, BLOCK, "nf4", out=y)))
-        ops.append((f"gemv_4bit_dq_{K}x{N}", N * K // 2 + nb + 4 * s8.numel() + 2 * K + 4 * N,
-                    lambda K=K, N=N, p=p, q8=q8, s8=s8, xv=xv, bias=bias, y=y:
-                    b.gemv_4bit_dq(xv, p, q8, s8, N, K, bias, BLOCK, "nf4", G, out=y)))
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    ev = [(torch.cuda.Event(enable_timing=True, external=True),
-           torch.cuda.Event(enable_timing=True, external=True)) for _ in ops]
-    for _, _, f in ops:
-        f()
-    cap = torch.cuda.Stream(dev)
-    cap.wait_stream(torch.cuda.current_stream(dev))
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=cap):
-        for (_, _, f), (e0, e1) in zip(ops, ev):
-            flush.fill_(1)
-            e0.record(cap)
-            f()
-            e1.record(cap)
-    torch.cuda.synchronize(dev)
-    g.replay()
-    torch.cuda.synchronize(dev)
-    times = [[] for _ in ops]
-    for _ in range(max(3, min(steps, 20))):
-        g.replay()
-        torch.cuda.synchronize(dev)
-        for i, (e0, e1) in enumerate(ev):
-            times[i].append(e0.elapsed_time(e1))
-    del g
+    C = copies_for(5 * n)
+    srcs = [step.absmax] + [step.absmax.clone() for _ in range(C - 1)]
+    qs = [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(C)]
+    ss = [torch.empty((n + G - 1) // G, dtype=torch.float32, device=dev) for _ in range(C)]
+    backs = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(C)]
+    for i in range(C):
+        b.double_quant(srcs[i], G, out=(qs[i], ss[i]))
     out = {}
-    for (nm, nbytes, _), t in zip(ops, times):
-        us = statistics.median(t) * 1e3
-        gbs = nbytes / (us / 1e6) / 1e9
-        out[nm] = {"us": round(us, 2), "bytes": nbytes, "GB/s": round(gbs, 1),
-                   "hbm_frac": round(gbs / hbm, 4)}
-    for K, N, *_ in step.gemv:
+
+    def rec(name, us, nbytes):
+        out[name] = {"us": round(us, 2), "bytes": int(nbytes), "GB/s": round(nbytes / (us / 1e6) / 1e9, 1),
+                     "hbm_frac": round(nbytes / (us / 1e6) / 1e9 / hbm, 4)}
+
+    rec("double_quant_absmax_4194304",
+        graph_per_launch(dev, [lambda i=i: b.double_quant(srcs[i], G, out=(qs[i], ss[i])) for i in range(C)]),
+        4 * n + n + 4 * ss[0].numel())
+    rec("dequant_absmax_4194304",
+        graph_per_launch(dev, [lambda i=i: b.dequant_absmax(qs[i], ss[i], G, out=backs[i]) for i in range(C)]),
+        n + 4 * ss[0].numel() + 4 * n)
+    del srcs, qs, ss, backs
+    for K, N, p, a, xv, bias, y in step.gemv:
+        nb = N * K // BLOCK
+        C = copies_for(N * K // 2 + 4 * nb)
+        ps = [p] + [p.clone() for _ in range(C - 1)]
+        as_ = [a] + [a.clone() for _ in range(C - 1)]
+        q8s, s8s = zip(*[b.double_quant(a_, G) for a_ in as_])
+        rec(f"gemv_4bit_{K}x{N}", graph_per_launch(dev, [
+            lambda i=i: b.gemv_4bit(xv, ps[i], as_[i], N, K, bias, BLOCK, "nf4", out=y) for i in range(C)]),
+            N * K // 2 + 4 * nb + 2 * K + 4 * N)
+        rec(f"gemv_4bit_dq_{K}x{N}", graph_per_launch(dev, [
+            lambda i=i: b.gemv_4bit_dq(xv, ps[i], q8s[i], s8s[i], N, K, bias, BLOCK, "nf4", G, out=y)
+            for i in range(C)]), N * K // 2 + nb + 4 * s8s[0].numel() + 2 * K + 4 * N)
         out[f"gemv_4bit_dq_{K}x{N}"]["speedup_vs_fp32_absmax"] = round(
             out[f"gemv_4bit_{K}x{N}"]["us"] / out[f"gemv_4bit_dq_{K}x{N}"]["us"], 3)
-    out["note"] = ("L2 flushed before each op; median of the replays; each time includes the "
-                   "few us of its two event nodes")
+        del ps, as_, q8s, s8s
+    out["note"] = ("each op alone, back to back in one CUDA graph over rotating copies of its inputs "
+                   "(working set above 5x L2)")
     return out
 
 
@@ -445,53 +590,48 @@ def code8_table(seed: int = 0):
     return torch.tensor(sorted(vals), dtype=torch.float32)
 
 
-def time_8bit_and_embedding(dev, reps, hbm):
-    """Rows f3 and f4 outside the step, L2 flushed before each op (median):
-    quantize_8bit / dequantize_8bit of 2^26 bf16 elements (B 64), and 4096
-    embedding lookups in a 128256 x 4096 NF4 table (B 64) to bf16."""
+def time_8bit_and_embedding(dev, hbm):
+    """Rows f3 and f4 outside the step: quantize_8bit / dequantize_8bit of 2^26
+    bf16 elements (B 64, a seeded log-spread table), and 4096 embedding lookups
+    in a 128256 x 4096 NF4 table (B 64) to bf16.  Each op timed with
+    graph_per_launch (the 8-bit inputs rotate over 3 copies, 600 MB; the
+    lookups read 43 MB of a 263 MB table at random rows)."""
     import bit_blockwise_weight_b200 as b
     import synthetic
     d = str(dev)
     n = 1 << 26
     code = code8_table(0)
-    x = synthetic.roundtrip_tensor(n, 0, "bf16", device=d)
-    q = torch.empty(n, dtype=torch.uint8, device=dev)
-    a8 = torch.empty(n // BLOCK, dtype=torch.float32, device=dev)
+    C = 3
+    xs = [synthetic.roundtrip_tensor(n, i, "bf16", device=d) for i in range(C)]
+    qs = [torch.empty(n, dtype=torch.uint8, device=dev) for _ in range(C)]
+    a8s = [torch.empty(n // BLOCK, dtype=torch.float32, device=dev) for _ in range(C)]
     y8 = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    stream = lambda: torch.cuda.current_stream(dev).cuda_stream
+    out = {}
+
+    def rec(name, us, nbytes):
+        out[name] = {"us": round(us, 2), "bytes": int(nbytes), "GB/s": round(nbytes / (us / 1e6) / 1e9, 1),
+                     "hbm_frac": round(nbytes / (us / 1e6) / 1e9 / hbm, 4)}
+
+    rec("quantize_8bit_2p26_bf16", graph_per_launch(dev, [
+        lambda i=i: b.bnb4_quantize_8bit(xs[i].data_ptr(), qs[i].data_ptr(), a8s[i].data_ptr(), n, BLOCK,
+                                         code.data_ptr(), 2, stream()) for i in range(C)]),
+        2 * n + n + 4 * (n // BLOCK))
+    rec("dequantize_8bit_2p26_bf16", graph_per_launch(dev, [
+        lambda i=i: b.bnb4_dequantize_8bit(qs[i].data_ptr(), a8s[i].data_ptr(), y8.data_ptr(), n, BLOCK,
+                                           code.data_ptr(), 2, stream()) for i in range(C)]),
+        n + 4 * (n // BLOCK) + 2 * n)
+    del xs, qs, a8s, y8
     V, D, T = 128256, 4096, 4096
     w = synthetic.normal((V * D,), 7, 0.02, "f32", device=d)
     ep, ea = b.quantize_4bit(w, BLOCK, "nf4")
     del w
     g = torch.Generator(device=d).manual_seed(11)
-    idx = torch.randint(0, V, (T,), generator=g, device=d, dtype=torch.int64)
+    idxs = [torch.randint(0, V, (T,), generator=g, device=d, dtype=torch.int64) for _ in range(8)]
     eo = torch.empty(T, D, dtype=torch.bfloat16, device=dev)
-    ops = [("quantize_8bit_2p26_bf16", 2 * n + n + 4 * (n // BLOCK),
-            lambda: b.bnb4_quantize_8bit(x.data_ptr(), q.data_ptr(), a8.data_ptr(), n, BLOCK, code.data_ptr(), 2,
-                                         torch.cuda.current_stream(dev).cuda_stream)),
-           ("dequantize_8bit_2p26_bf16", n + 4 * (n // BLOCK) + 2 * n,
-            lambda: b.bnb4_dequantize_8bit(q.data_ptr(), a8.data_ptr(), y8.data_ptr(), n, BLOCK, code.data_ptr(), 2,
-                                           torch.cuda.current_stream(dev).cuda_stream)),
-           ("embedding_4bit_4096_of_128256x4096", T * (D // 2 + 4 * (D // BLOCK)) + 8 * T + 2 * T * D,
-            lambda: b.embedding_4bit(ep, ea, V, D, idx, BLOCK, "nf4", out=eo))]
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-    for _, _, f in ops:
-        f()
-    torch.cuda.synchronize(dev)
-    times = [[] for _ in ops]
-    for _ in range(max(3, reps)):
-        for i, (_, _, f) in enumerate(ops):
-            flush.fill_(1)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            f()
-            e1.record()
-            torch.cuda.synchronize(dev)
-            times[i].append(e0.elapsed_time(e1))
-    out = {}
-    for (nm, nbytes, _), t in zip(ops, times):
-        us = statistics.median(t) * 1e3
-        out[nm] = {"us": round(us, 2), "bytes": nbytes, "GB/s": round(nbytes / (us / 1e6) / 1e9, 1),
-                   "hbm_frac": round(nbytes / (us / 1e6) / 1e9 / hbm, 4)}
+    rec("embedding_4bit_4096_of_128256x4096", graph_per_launch(dev, [
+        lambda i=i: b.embedding_4bit(ep, ea, V, D, idxs[i], BLOCK, "nf4", out=eo) for i in range(8)]),
+        T * (D // 2 + 4 * (D // BLOCK)) + 8 * T + 2 * T * D)
     return out
 
 

@@ -144,7 +144,10 @@ bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, cons
                       bnb4_dtype dt, cudaStream_t stream) {
     bnb4_status s = check_matmul(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt);
     if (s != BNB4_OK) return s;
-    // small M: one pass over the weight stream, decoded into tensor memory
+    // one token: the gemv kernel (the same product, faster at M == 1)
+    if (M == 1 && N <= gemv_max_rows() && K <= gemv_max_k())
+        return from_cuda(launch_gemv(X, W, absmax, nullptr, nullptr, 0, bias, Y, N, K, blocksize, qt, dt, stream));
+    // small M: one pass over the weight stream, tensor-core tiles fed from registers
     if (M <= kSmallMMax)
         return from_cuda(launch_gemm_small(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, stream));
     return from_cuda(launch_gemm_tc(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, false, stream));

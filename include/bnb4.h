@@ -168,9 +168,10 @@ bnb4_status bnb4_gemv_dq(const void *x, const uint8_t *packedW,
 /*
  * General matmul: Y[M, N] = X[M, K] @ dequant(W)^T (+ bias), row-major.
  *   X [M, K] of dt;  bias [N] of dt or NULL;  Y [M, N] of dt (out).
- *   Same constraints as bnb4_gemv; M >= 1.  Small M streams the weight once
- *   through a register-decode tensor-core kernel, large M runs the tcgen05
- *   kernel that dequantizes weight tiles into shared memory.
+ *   Same constraints as bnb4_gemv; M >= 1.  M == 1 runs the gemv kernel,
+ *   small M streams the weight once through a register-decode tensor-core
+ *   kernel, large M runs the tcgen05 kernel that dequantizes weight tiles
+ *   into shared memory.
  */
 bnb4_status bnb4_gemm(const void *X, const uint8_t *packedW,
                       const float *absmax, const void *bias, void *Y,

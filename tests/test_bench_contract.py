@@ -23,16 +23,19 @@ def test_step_ops_cover_every_launch_once():
 def test_roofline_and_parts():
     ops = [("quantize_4bit", 6_000_000, 0), ("gemm_4bit_M512_4096x14336", 40_000_000, 60_129_542_144),
            ("gemv_4bit_4096x4096", 9_000_000, 33_554_432)]
-    roof, parts = bench.roofline_and_parts(ops, [0.002, 0.080, 0.010], 6500.0, 1400.0, "measured",
+    roof, parts = bench.roofline_and_parts(ops, [0.002, 0.080, 0.010], 6500.0, 1683.5, 1400.0, "measured",
                                            traffic=lambda name: 123)
-    # the tensor-core op has the largest share: TFLOP/s against the sustained peak
+    # the tensor-core op has the largest share: TFLOP/s against the burst peak,
+    # the sustained fraction beside it
     assert roof["bound"] == "tensor" and roof["kernel"] == "gemm_4bit_M512_4096x14336"
     assert roof["achieved"] == pytest.approx(60_129_542_144 / 80e-6 / 1e12, abs=0.1)
-    assert roof["frac"] == pytest.approx(roof["achieved"] / 1400.0, abs=1e-4)
+    assert roof["peak"] == 1683.5
+    assert roof["frac"] == pytest.approx(roof["achieved"] / 1683.5, abs=1e-4)
+    assert roof["frac_of_sustained"] == pytest.approx(roof["achieved"] / 1400.0, abs=1e-4)
     assert roof["traffic"] == 123 and roof["unit"] == "TFLOP/s"
     assert sum(p["share"] for p in parts.values()) == pytest.approx(1.0, abs=1e-3)
     assert parts["quantize_4bit"]["GB/s"] == pytest.approx(6e6 / 2e-6 / 1e9, abs=0.1)
-    roof, _ = bench.roofline_and_parts(ops[:1] + ops[2:], [0.5, 0.01], 6500.0, 1400.0, "measured",
+    roof, _ = bench.roofline_and_parts(ops[:1] + ops[2:], [0.5, 0.01], 6500.0, 1683.5, 1400.0, "measured",
                                        traffic=lambda name: None)
     assert roof["bound"] == "hbm" and roof["peak"] == 6500.0 and roof["traffic"] is None
     assert roof["frac"] == pytest.approx(6e6 / 0.5e-3 / 1e9 / 6500.0, abs=1e-4)

@@ -40,14 +40,14 @@ constexpr int64_t kMaxDim = (int64_t)1 << 31;
 
 bnb4_status check_matmul(const void *a, const uint8_t *W, const float *absmax, const void *bias,
                          const void *out, int64_t M, int64_t N, int64_t K, int blocksize,
-                         bnb4_quant_type qt, bnb4_dtype dt) {
+                         bnb4_quant_type qt, bnb4_dtype dt, bool allow_f32) {
     if (!a || !W || !absmax || !out) return BNB4_ERR_NULL;
     if (!aligned16(a) || !aligned16(W) || !aligned16(absmax) || !aligned16(out) ||
         (bias && !aligned16(bias)))
         return BNB4_ERR_ALIGN;
     if (!valid_blocksize(blocksize)) return BNB4_ERR_BLOCKSIZE;
     if (!valid_qtype(qt)) return BNB4_ERR_QTYPE;
-    if (dt != BNB4_F16 && dt != BNB4_BF16) return BNB4_ERR_DTYPE;
+    if (dt != BNB4_F16 && dt != BNB4_BF16 && !(allow_f32 && dt == BNB4_F32)) return BNB4_ERR_DTYPE;
     if (M < 1 || N < 1 || K < 1 || M >= kMaxDim || N >= kMaxDim || K >= kMaxDim)
         return BNB4_ERR_SHAPE;
     if (K % 32 != 0 || K % blocksize != 0) return BNB4_ERR_SHAPE;
@@ -113,8 +113,9 @@ bnb4_status bnb4_dequantize(const uint8_t *packed, const float *absmax, void *ou
 bnb4_status bnb4_gemv(const void *x, const uint8_t *W, const float *absmax, const void *bias,
                       void *y, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
                       bnb4_dtype dt, cudaStream_t stream) {
-    bnb4_status s = check_matmul(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt);
+    bnb4_status s = check_matmul(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt, true);
     if (s != BNB4_OK) return s;
+    if (dt == BNB4_F32) return bnb4_gemm(x, W, absmax, bias, y, 1, N, K, blocksize, qt, dt, stream);
     if (N <= gemv_max_rows() && K <= gemv_max_k())
         return from_cuda(launch_gemv(x, W, absmax, nullptr, nullptr, 0, bias, y, N, K, blocksize, qt, dt,
                                      stream));
@@ -131,7 +132,7 @@ bnb4_status bnb4_gemv_dq(const void *x, const uint8_t *W, const uint8_t *absmax_
     if (!aligned16(absmax_scales)) return BNB4_ERR_ALIGN;
     // absmax_q stands in the fp32 absmax's place for the common checks
     bnb4_status s = check_matmul(x, W, reinterpret_cast<const float *>(absmax_q), bias, y, 1, N, K,
-                                 blocksize, qt, dt);
+                                 blocksize, qt, dt, false);
     if (s != BNB4_OK) return s;
     if (group < 32 || group > 4096 || (group & (group - 1)) != 0) return BNB4_ERR_BLOCKSIZE;
     if (N > gemv_max_rows() || K > gemv_max_k()) return BNB4_ERR_SHAPE;
@@ -142,8 +143,17 @@ bnb4_status bnb4_gemv_dq(const void *x, const uint8_t *W, const uint8_t *absmax_
 bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, const void *bias,
                       void *Y, int64_t M, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
                       bnb4_dtype dt, cudaStream_t stream) {
-    bnb4_status s = check_matmul(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt);
+    bnb4_status s = check_matmul(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, true);
     if (s != BNB4_OK) return s;
+    if (dt == BNB4_F32) {
+        // fp32: CUDA-core kernels with the exact fp32 dequantized weight
+        if (M == 1 && N <= gemv_f32_max_rows() && K <= gemv_f32_max_k())
+            return from_cuda(launch_gemv_f32(static_cast<const float *>(X), W, absmax,
+                                             static_cast<const float *>(bias), static_cast<float *>(Y), N, K,
+                                             blocksize, qt, stream));
+        return from_cuda(launch_gemm_f32(static_cast<const float *>(X), W, absmax, static_cast<const float *>(bias),
+                                         static_cast<float *>(Y), M, N, K, blocksize, qt, false, stream));
+    }
     // one token: the gemv kernel (the same product, faster at M == 1)
     if (M == 1 && N <= gemv_max_rows() && K <= gemv_max_k())
         return from_cuda(launch_gemv(X, W, absmax, nullptr, nullptr, 0, bias, Y, N, K, blocksize, qt, dt, stream));
@@ -156,8 +166,11 @@ bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, cons
 bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *absmax, void *dX,
                                int64_t M, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt,
                                bnb4_dtype dt, cudaStream_t stream) {
-    bnb4_status s = check_matmul(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt);
+    bnb4_status s = check_matmul(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true);
     if (s != BNB4_OK) return s;
+    if (dt == BNB4_F32)
+        return from_cuda(launch_gemm_f32(static_cast<const float *>(dY), W, absmax, nullptr, static_cast<float *>(dX),
+                                         M, N, K, blocksize, qt, true, stream));
     if (N % 8 != 0) return BNB4_ERR_SHAPE;  // dY rows are TMA-loaded: 16-byte row pitch
     return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true, stream));
 }

@@ -1,0 +1,325 @@
+// gemm_f32.cu -- the 4-bit matmuls in fp32: x, bias and y in float32, and the
+// weight a product meets is the exact fp32 dequantized value RN32(code *
+// absmax) ("Feat/mps gemm 4bit bf16", Performance: gemv_4bit is measured
+// across fp16, bf16 and fp32).  Products and sums are fp32 FMAs on the CUDA
+// cores: the tensor cores' fp32 input path (tf32) keeps 10 mantissa bits,
+// which this dtype's accuracy rules out.
+//
+//   gemv_f32_kernel   M == 1.  CTA c owns rows [N c / G, N (c+1) / G) and all
+//                     of K; its work is a list of units (a quad of rows x 1024
+//                     weights of K), quad major, split into contiguous,
+//                     balanced ranges, one per warp.  Lane l holds 32
+//                     consecutive weights of each row of the unit (16-byte
+//                     loads, one group of loads ahead of the arithmetic) and
+//                     the matching 32 values of x, read once from shared
+//                     memory for the four rows.  Each code comes from a
+//                     16-entry table replicated once per bank (conflict-free),
+//                     is multiplied by its block's absmax (the exact fp32
+//                     weight) and accumulated with an FMA.  Row sums are
+//                     reduced across lanes when a warp leaves a quad; quads
+//                     that two warps share are added in warp order, so the
+//                     result is the same bits on every run.
+//   gemm_f32_kernel   M >= 2 and the backward.  A classic shared-memory tiled
+//                     product: BM x 64 output tiles, 64-wide reduction steps;
+//                     the step's weight tile is dequantized into shared memory
+//                     as fp32 (transposed for the forward, as stored for the
+//                     backward), the activations tile is staged beside it,
+//                     and each thread accumulates a 4 x 4 (BM = 64) or 1 x 4
+//                     (BM = 16) block of outputs.
+//
+// No global scratch.
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bnb4 {
+
+namespace {
+
+// ------------------------------------------------------------------ gemv
+
+constexpr int kVWarps = 16;
+constexpr int kVThreads = kVWarps * 32;
+constexpr int kVUnitK = 1024;                 // weights per row per unit (32 lanes x 32)
+constexpr int kVMaxRows = 1024;               // rows per CTA
+constexpr int kVMaxK = 32768;
+
+__device__ __forceinline__ uint4 ldg_nc16(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__global__ void __launch_bounds__(kVThreads, 1)
+gemv_f32_kernel(const float *__restrict__ x, const uint8_t *__restrict__ W, const float *__restrict__ absmax,
+                const float *__restrict__ bias, float *__restrict__ y, int N, int K, int log2B,
+                const __grid_constant__ CodeTable tab) {
+    extern __shared__ __align__(16) float vsm[];
+    float *code = vsm;                                 // [16][32]: entry e, copy l at 32 e + l
+    float *rowsum = code + 16 * 32;                    // [kVMaxRows]
+    float *part = rowsum + kVMaxRows;                  // [kVWarps][2][4]
+    float *xs = part + kVWarps * 8;                    // [K rounded up to kVUnitK]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = gridDim.x;
+    const int r0 = (int)(((int64_t)N * blockIdx.x) / G);
+    const int r1 = (int)(((int64_t)N * (blockIdx.x + 1)) / G);
+    const int R = r1 - r0;
+    const int NQ = (R + 3) >> 2;
+    const int S = (K + kVUnitK - 1) / kVUnitK;         // units per quad
+    const int GU = NQ * S;
+    const int u_lo = (int)(((int64_t)GU * warp) / kVWarps);
+    const int u_hi = (int)(((int64_t)GU * (warp + 1)) / kVWarps);
+    const int64_t row_bytes = K >> 1;
+    const int nblk = K >> log2B;
+
+    for (int i = tid; i < 16 * 32; i += kVThreads) code[i] = tab.v[i >> 5];
+    const int Kp = S * kVUnitK;
+    for (int i = tid; i < Kp / 4; i += kVThreads)
+        reinterpret_cast<float4 *>(xs)[i] = 4 * i < K ? __ldg(reinterpret_cast<const float4 *>(x) + i)
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+
+    // the lane's 32 weights of each row of unit (q, s): rows past the CTA's
+    // last row are clamped to it (their sums are never stored), weights past
+    // K are clamped in place (they meet zeros of x)
+    struct Rows {
+        uint4 w[4];
+        float a[4];
+    };
+    auto load = [&](int u, Rows &rw) {
+        const int q = u / S, s = u - q * S;
+        const int k = min(s * kVUnitK + 32 * lane, K - 32);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int rl = min(4 * q + r, R - 1);
+            const int64_t row = r0 + rl;
+            rw.w[r] = ldg_nc16(W + row * row_bytes + (k >> 1));
+            rw.a[r] = __ldg(absmax + row * nblk + (k >> log2B));
+        }
+    };
+
+    Rows cur, nxt;
+    if (u_lo < u_hi) load(u_lo, cur);
+    __syncthreads();
+
+    const int q_first = u_lo < u_hi ? u_lo / S : -1;
+    const int q_last = u_lo < u_hi ? (u_hi - 1) / S : -1;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int u = u_lo; u < u_hi; ++u) {
+        if (u + 1 < u_hi) load(u + 1, nxt);
+        const int q = u / S, s = u - q * S;
+        const int k = s * kVUnitK + 32 * lane;
+        float xv[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 v = reinterpret_cast<const float4 *>(xs + k)[i];
+            xv[4 * i] = v.x;
+            xv[4 * i + 1] = v.y;
+            xv[4 * i + 2] = v.z;
+            xv[4 * i + 3] = v.w;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const uint32_t w4[4] = {cur.w[r].x, cur.w[r].y, cur.w[r].z, cur.w[r].w};
+            float sacc = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t b = (w4[i >> 2] >> (8 * (i & 3))) & 255u;
+                // first element of the byte in its high nibble; the exact weight RN32(code * absmax)
+                const float w0 = __fmul_rn(code[((b >> 4) << 5) + lane], cur.a[r]);
+                const float w1 = __fmul_rn(code[((b & 15u) << 5) + lane], cur.a[r]);
+                sacc = __fmaf_rn(xv[2 * i], w0, sacc);
+                sacc = __fmaf_rn(xv[2 * i + 1], w1, sacc);
+            }
+            acc[r] += sacc;
+        }
+        if (u + 1 == u_hi || (u + 1) / S != q) {
+            // reduce the 4 row sums over the 32 lanes: halve over bits 4 and 3,
+            // then plain sums over bits 2, 1, 0; lanes 0, 8, 16, 24 end with rows 0..3
+            const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0;
+            float k0 = b4 ? acc[2] : acc[0], k1 = b4 ? acc[3] : acc[1];
+            k0 += __shfl_xor_sync(FULL, b4 ? acc[0] : acc[2], 16);
+            k1 += __shfl_xor_sync(FULL, b4 ? acc[1] : acc[3], 16);
+            float v = b3 ? k1 : k0;
+            v += __shfl_xor_sync(FULL, b3 ? k0 : k1, 8);
+            v += __shfl_xor_sync(FULL, v, 4);
+            v += __shfl_xor_sync(FULL, v, 2);
+            v += __shfl_xor_sync(FULL, v, 1);
+            if ((lane & 7) == 0) {
+                const int rr = 2 * (int)b4 + (int)b3;
+                if (q == q_first) part[warp * 8 + rr] = v;
+                else if (q == q_last) part[warp * 8 + 4 + rr] = v;
+                else if (4 * q + rr < R) rowsum[4 * q + rr] = v;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[r] = 0.f;
+        }
+        if (u + 1 < u_hi) cur = nxt;
+    }
+    __syncthreads();
+    for (int r = tid; r < R; r += kVThreads) {
+        const int q = r >> 2, rr = r & 3, ul = q * S, uh = ul + S;
+        const int w0 = (kVWarps * (ul + 1) + GU - 1) / GU - 1, w1 = (kVWarps * uh + GU - 1) / GU - 1;
+        float v = 0.f;
+        for (int w = w0; w <= w1; ++w) {
+            const int lo = (int)(((int64_t)GU * w) / kVWarps), hi = (int)(((int64_t)GU * (w + 1)) / kVWarps);
+            if (lo >= hi) continue;
+            v += lo >= ul ? part[w * 8 + rr] : hi - 1 < uh ? part[w * 8 + 4 + rr] : rowsum[r];
+        }
+        if (bias) v += bias[r0 + r];
+        y[r0 + r] = v;
+    }
+}
+
+// -------------------------------------------------------------- tiled gemm
+
+constexpr int kBN = 64;   // output columns per tile (weight rows forward, K columns backward)
+constexpr int kBK = 64;   // reduction step
+constexpr int kGThreads = 256;
+
+// BWD == false: Y[m, n] = sum_k A[m, k] W[n, k] (+ bias[n]), A = X [M, K], tile over (m, n), step over k.
+// BWD == true:  Y[m, k] = sum_n A[m, n] W[n, k], A = dY [M, N], tile over (m, k), step over n.
+template <int BM, bool BWD>
+__global__ void __launch_bounds__(kGThreads)
+gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, const float *__restrict__ absmax,
+                const float *__restrict__ bias, float *__restrict__ Y, int M, int N, int K, int log2B,
+                const __grid_constant__ CodeTable tab) {
+    constexpr int TM = BM / 16;                    // outputs per thread along m (4 or 1)
+    __shared__ __align__(16) float As[kBK][BM + 4];     // [reduction][m]
+    __shared__ __align__(16) float Bs[kBK][kBN + 4];    // [reduction][output column]
+    __shared__ float code[16];
+    const int tid = threadIdx.x;
+    if (tid < 16) code[tid] = tab.v[tid];
+    const int m0 = blockIdx.y * BM;
+    const int c0 = blockIdx.x * kBN;               // first output column of the tile
+    const int ncols = BWD ? K : N;                 // output columns
+    const int red = BWD ? N : K;                   // reduction length
+    const int tx = tid & 15, ty = tid >> 4;        // 16 x 16 threads: columns 4 tx.., rows TM ty..
+    const int64_t row_bytes = K >> 1;
+    const int nblk = K >> log2B;
+    float acc[TM][4];
+#pragma unroll
+    for (int i = 0; i < TM; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    __syncthreads();
+
+    for (int r0 = 0; r0 < red; r0 += kBK) {
+        // activations: A[m0 + i][r0 + j] -> As[j][i], zeros outside
+        for (int e = tid; e < BM * kBK; e += kGThreads) {
+            const int i = e / kBK, j = e % kBK;
+            const int m = m0 + i, r = r0 + j;
+            As[j][i] = (m < M && r < red) ? A[(int64_t)m * red + r] : 0.f;
+        }
+        // weight tile: 64 weight rows x 64 weights, one thread per (row, 16 weights)
+        {
+            const int lr = tid >> 2, part = tid & 3;   // tile row, quarter of the 64 weights
+            int wrow, wk;                               // weight row and first k of this thread's 16
+            if (!BWD) { wrow = c0 + lr; wk = r0 + 16 * part; }
+            else { wrow = r0 + lr; wk = c0 + 16 * part; }
+            float v[16];
+            if (wrow < N && wk < K) {
+                const uint2 p = __ldg(reinterpret_cast<const uint2 *>(W + (int64_t)wrow * row_bytes + (wk >> 1)));
+                const float a = __ldg(absmax + (int64_t)wrow * nblk + (wk >> log2B));
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t b = ((i < 4 ? p.x : p.y) >> (8 * (i & 3))) & 255u;
+                    v[2 * i] = __fmul_rn(code[b >> 4], a);
+                    v[2 * i + 1] = __fmul_rn(code[b & 15u], a);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                if (!BWD) Bs[16 * part + i][lr] = v[i];       // [k][n]
+                else Bs[lr][16 * part + i] = v[i];            // [n][k]
+            }
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int j = 0; j < kBK; ++j) {
+            float a[TM];
+#pragma unroll
+            for (int i = 0; i < TM; ++i) a[i] = As[j][TM * ty + i];
+            const float4 bq = *reinterpret_cast<const float4 *>(&Bs[j][4 * tx]);
+            const float b[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[i][c] = __fmaf_rn(a[i], b[c], acc[i][c]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < TM; ++i) {
+        const int m = m0 + TM * ty + i;
+        if (m >= M) continue;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int col = c0 + 4 * tx + c;
+            if (col >= ncols) continue;
+            float v = acc[i][c];
+            if (!BWD && bias) v += bias[col];
+            Y[(int64_t)m * ncols + col] = v;
+        }
+    }
+}
+
+size_t gemv_f32_smem(int K) {
+    const size_t Kp = ((size_t)K + kVUnitK - 1) / kVUnitK * kVUnitK;
+    return (16 * 32 + kVMaxRows + kVWarps * 8 + Kp) * sizeof(float);
+}
+
+}  // namespace
+
+int64_t gemv_f32_max_rows() { return (int64_t)device_sm_count() * kVMaxRows; }
+int64_t gemv_f32_max_k() { return kVMaxK; }
+
+cudaError_t launch_gemv_f32(const float *x, const uint8_t *W, const float *absmax, const float *bias, float *y,
+                            int64_t N, int64_t K, int blocksize, bnb4_quant_type qt, cudaStream_t stream) {
+    static const CodeTable nf4 = host_code_table(BNB4_NF4);
+    static const CodeTable fp4 = host_code_table(BNB4_FP4);
+    const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
+    static std::atomic<bool> set[kMaxDevices];
+    cudaError_t e = once_per_device(set, [] {
+        return cudaFuncSetAttribute(gemv_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)gemv_f32_smem(kVMaxK));
+    });
+    if (e != cudaSuccess) return e;
+    gemv_f32_kernel<<<device_sm_count(), kVThreads, gemv_f32_smem((int)K), stream>>>(
+        x, W, absmax, bias, y, (int)N, (int)K, ilog2(blocksize), tab);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_f32(const float *A, const uint8_t *W, const float *absmax, const float *bias, float *Y,
+                            int64_t M, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt, bool backward,
+                            cudaStream_t stream) {
+    static const CodeTable nf4 = host_code_table(BNB4_NF4);
+    static const CodeTable fp4 = host_code_table(BNB4_FP4);
+    const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
+    const int ncols = (int)(backward ? K : N);
+    const int log2B = ilog2(blocksize);
+    if (M <= 16) {
+        const dim3 grid((ncols + kBN - 1) / kBN, (unsigned)((M + 15) / 16));
+        if (backward)
+            gemm_f32_kernel<16, true><<<grid, kGThreads, 0, stream>>>(A, W, absmax, nullptr, Y, (int)M, (int)N,
+                                                                     (int)K, log2B, tab);
+        else
+            gemm_f32_kernel<16, false><<<grid, kGThreads, 0, stream>>>(A, W, absmax, bias, Y, (int)M, (int)N,
+                                                                      (int)K, log2B, tab);
+    } else {
+        const dim3 grid((ncols + kBN - 1) / kBN, (unsigned)((M + 63) / 64));
+        if (backward)
+            gemm_f32_kernel<64, true><<<grid, kGThreads, 0, stream>>>(A, W, absmax, nullptr, Y, (int)M, (int)N,
+                                                                     (int)K, log2B, tab);
+        else
+            gemm_f32_kernel<64, false><<<grid, kGThreads, 0, stream>>>(A, W, absmax, bias, Y, (int)M, (int)N,
+                                                                      (int)K, log2B, tab);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace bnb4

@@ -44,6 +44,17 @@ cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax,
                            int blocksize, bnb4_quant_type qt, bnb4_dtype dt, bool backward,
                            cudaStream_t stream);
 
+// fp32 compute dtype (x, bias, y in float32; the exact fp32 dequantized
+// weight; CUDA-core FMAs): M == 1 up to gemv_f32_max_rows() x gemv_f32_max_k(),
+// and a tiled kernel for any M (backward == true computes dX = dY @ dequant(W))
+int64_t gemv_f32_max_rows();
+int64_t gemv_f32_max_k();
+cudaError_t launch_gemv_f32(const float *x, const uint8_t *W, const float *absmax, const float *bias, float *y,
+                            int64_t N, int64_t K, int blocksize, bnb4_quant_type qt, cudaStream_t stream);
+cudaError_t launch_gemm_f32(const float *A, const uint8_t *W, const float *absmax, const float *bias, float *Y,
+                            int64_t M, int64_t N, int64_t K, int blocksize, bnb4_quant_type qt, bool backward,
+                            cudaStream_t stream);
+
 // double quantization of an absmax array (groups of `group`, a power of two
 // in [32, 4096]) and its inverse
 cudaError_t launch_double_quant(const float *absmax, int64_t n, int group, uint8_t *q, float *scales,

@@ -31,8 +31,8 @@ int main(void) {
            "dequantize null out");
     expect(bnb4_gemv(a, (const uint8_t *)a, (const float *)a, 0, a, 64, 100, 64, BNB4_NF4, BNB4_BF16, 0),
            BNB4_ERR_SHAPE, "gemv K%32");
-    expect(bnb4_gemm(a, (const uint8_t *)a, (const float *)a, 0, a, 2, 64, 128, 64, BNB4_NF4, BNB4_F32, 0),
-           BNB4_ERR_DTYPE, "gemm f32");
+    expect(bnb4_gemm(a, (const uint8_t *)a, (const float *)a, 0, a, 2, 64, 128, 64, BNB4_NF4, (bnb4_dtype)7, 0),
+           BNB4_ERR_DTYPE, "gemm dtype");
     expect(bnb4_gemm_backward(a, (const uint8_t *)a, (const float *)a, a, 2, 60, 128, 64, BNB4_NF4, BNB4_BF16, 0),
            BNB4_ERR_SHAPE, "backward N%8");
     expect(bnb4_double_quant((const float *)a, 10, 100, (uint8_t *)a, (float *)a, 0), BNB4_ERR_BLOCKSIZE,

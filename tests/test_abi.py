@@ -75,7 +75,8 @@ def test_matmul_argument_checks():
     assert g(A, A, A, None, A, 128, 100, 64, 0, 2, None) == 4   # K % 32
     assert g(A, A, A, None, A, 128, 96, 64, 0, 2, None) == 4    # K % blocksize
     assert g(A, A, A, None, A, 0, 128, 64, 0, 2, None) == 4     # N < 1
-    assert g(A, A, A, None, A, 128, 128, 64, 0, 0, None) == 5   # f32 not a compute dtype
+    assert g(A, A, A, None, A, 128, 128, 64, 0, 7, None) == 5   # not a dtype
+    assert bnb4.bnb4_gemv_dq(A, A, A, A, 256, None, A, 128, 128, 64, 0, 0, None) == 5  # no f32 on 8-bit statistics
     assert g(A, A, A, A + 4, A, 128, 128, 64, 0, 2, None) == 2  # misaligned bias
     assert g(A, None, A, None, A, 128, 128, 64, 0, 2, None) == 1
     m = bnb4.bnb4_gemm

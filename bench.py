@@ -572,8 +572,38 @@ def time_next_rows(step, dev, hbm):
         out[f"gemv_4bit_dq_{K}x{N}"]["speedup_vs_fp32_absmax"] = round(
             out[f"gemv_4bit_{K}x{N}"]["us"] / out[f"gemv_4bit_dq_{K}x{N}"]["us"], 3)
         del ps, as_, q8s, s8s
+    # M >= 2 on 8-bit statistics: small-M M = 16 on the 70B shapes and prefill M = 512
+    # forward / backward, each beside the same op on fp32 absmax
+    for K, N, p, a, X, Y in step.smallm:
+        q8, s8 = b.double_quant(a, G)
+        nb = N * K // BLOCK
+        ps = [p, p.clone()]
+        as_ = [a, a.clone()]
+        q8s, s8s = [q8, q8.clone()], [s8, s8.clone()]
+        M = X.shape[0]
+        rec(f"gemm_4bit_M{M}_{K}x{N}", graph_per_launch(dev, [
+            lambda i=i: b.gemm_4bit(X, ps[i], as_[i], N, None, BLOCK, "nf4", out=Y) for i in range(2)]),
+            N * K // 2 + 4 * nb + 2 * M * K + 2 * M * N)
+        rec(f"gemm_4bit_dq_M{M}_{K}x{N}", graph_per_launch(dev, [
+            lambda i=i: b.gemm_4bit_dq(X, ps[i], q8s[i], s8s[i], N, None, BLOCK, "nf4", G, out=Y) for i in range(2)]),
+            N * K // 2 + nb + 4 * s8.numel() + 2 * M * K + 2 * M * N)
+        out[f"gemm_4bit_dq_M{M}_{K}x{N}"]["speedup_vs_fp32_absmax"] = round(
+            out[f"gemm_4bit_M{M}_{K}x{N}"]["us"] / out[f"gemm_4bit_dq_M{M}_{K}x{N}"]["us"], 3)
+        del ps, as_, q8s, s8s
+    M, K, N, p, a, X, dY, Y, dX = step.prefill
+    q8, s8 = b.double_quant(a, G)
+    for name, f32f, dqf in (
+            (f"gemm_4bit_M{M}_{K}x{N}", lambda: b.gemm_4bit(X, p, a, N, None, BLOCK, "nf4", out=Y),
+             lambda: b.gemm_4bit_dq(X, p, q8, s8, N, None, BLOCK, "nf4", G, out=Y)),
+            (f"gemm_4bit_backward_M{M}_{K}x{N}", lambda: b.gemm_4bit_backward(dY, p, a, K, BLOCK, "nf4", out=dX),
+             lambda: b.gemm_4bit_backward_dq(dY, p, q8, s8, K, BLOCK, "nf4", G, out=dX))):
+        t32 = graph_per_launch(dev, [f32f] * 4)
+        tdq = graph_per_launch(dev, [dqf] * 4)
+        out[name] = {"us": round(t32, 2)}
+        dqn = name.replace("gemm_4bit", "gemm_4bit_dq", 1)
+        out[dqn] = {"us": round(tdq, 2), "speedup_vs_fp32_absmax": round(t32 / tdq, 3)}
     out["note"] = ("each op alone, back to back in one CUDA graph over rotating copies of its inputs "
-                   "(working set above 5x L2)")
+                   "(working set above 5x L2; the prefill ops reuse one 33 MB weight, compute-bound)")
     return out
 
 

@@ -4,7 +4,8 @@ Two layers, both argument marshalling only (every step of the computation
 runs in the library's CUDA kernels):
 
 * ``bnb4_quantize``, ``bnb4_dequantize``, ``bnb4_gemv``, ``bnb4_gemm``,
-  ``bnb4_gemm_backward``, ``bnb4_gemv_dq``, ``bnb4_double_quant``, ``bnb4_dequant_absmax``,
+  ``bnb4_gemm_backward``, ``bnb4_gemv_dq``, ``bnb4_gemm_dq``, ``bnb4_gemm_backward_dq``,
+  ``bnb4_double_quant``, ``bnb4_dequant_absmax``,
   ``bnb4_quantize_8bit``, ``bnb4_dequantize_8bit``, ``bnb4_embedding_4bit``,
   ``bnb4_device_status``, ``bnb4_selftest_wait_timeout``: the C ABI of
   ``include/bnb4.h`` one to one (raw
@@ -12,7 +13,7 @@ runs in the library's CUDA kernels):
   They return the integer status.
 * ``quantize_4bit``, ``dequantize_4bit``, ``gemv_4bit``, ``gemm_4bit``,
   ``gemm_4bit_backward``, ``double_quant``, ``dequant_absmax``,
-  ``gemv_4bit_dq``, ``quantize_8bit``, ``dequantize_8bit``,
+  ``gemv_4bit_dq``, ``gemm_4bit_dq``, ``gemm_4bit_backward_dq``, ``quantize_8bit``, ``dequantize_8bit``,
   ``embedding_4bit``, ``device_status``: take torch CUDA tensors (the 8-bit
   code table on the host), allocate outputs with torch, call the C ABI on the
   current stream and raise ``Bnb4Error`` on a non-OK status.
@@ -56,6 +57,8 @@ def _load() -> ctypes.CDLL:
         "bnb4_gemm": (I, [P, P, P, P, P, I64, I64, I64, I, I, I, P]),
         "bnb4_gemm_backward": (I, [P, P, P, P, I64, I64, I64, I, I, I, P]),
         "bnb4_gemv_dq": (I, [P, P, P, P, I, P, P, I64, I64, I, I, I, P]),
+        "bnb4_gemm_dq": (I, [P, P, P, P, I, P, P, I64, I64, I64, I, I, I, P]),
+        "bnb4_gemm_backward_dq": (I, [P, P, P, P, I, P, I64, I64, I64, I, I, I, P]),
         "bnb4_quantize_8bit": (I, [P, P, P, I64, I, P, I, P]),
         "bnb4_dequantize_8bit": (I, [P, P, P, I64, I, P, I, P]),
         "bnb4_embedding_4bit": (I, [P, P, I64, I64, I, I, P, I64, P, I, P]),
@@ -81,6 +84,8 @@ bnb4_gemv = _lib.bnb4_gemv
 bnb4_gemm = _lib.bnb4_gemm
 bnb4_gemm_backward = _lib.bnb4_gemm_backward
 bnb4_gemv_dq = _lib.bnb4_gemv_dq
+bnb4_gemm_dq = _lib.bnb4_gemm_dq
+bnb4_gemm_backward_dq = _lib.bnb4_gemm_backward_dq
 bnb4_quantize_8bit = _lib.bnb4_quantize_8bit
 bnb4_dequantize_8bit = _lib.bnb4_dequantize_8bit
 bnb4_embedding_4bit = _lib.bnb4_embedding_4bit
@@ -217,6 +222,31 @@ def gemm_4bit_backward(dY, packed, absmax, K: int, blocksize: int = 64, quant_ty
     _check(bnb4_gemm_backward(_ptr(dY), _ptr(packed), _ptr(absmax), _ptr(dX), M, N, K, blocksize,
                               _qtype(quant_type), _dtype_code(dY), _stream(stream)),
            "bnb4_gemm_backward")
+    return dX
+
+
+def gemm_4bit_dq(X, packed, absmax_q, absmax_scales, N: int, bias=None, blocksize: int = 64,
+                 quant_type="nf4", group: int = 256, out=None, stream=None):
+    """gemm_4bit with the absmax given as double_quant's (codes, scales)."""
+    torch = _torch()
+    _need_cuda(X, packed, absmax_q, absmax_scales, bias)
+    M, K = X.shape
+    Y = out if out is not None else torch.empty(M, N, dtype=X.dtype, device=X.device)
+    _check(bnb4_gemm_dq(_ptr(X), _ptr(packed), _ptr(absmax_q), _ptr(absmax_scales), group, _ptr(bias), _ptr(Y),
+                        M, N, K, blocksize, _qtype(quant_type), _dtype_code(X), _stream(stream)), "bnb4_gemm_dq")
+    return Y
+
+
+def gemm_4bit_backward_dq(dY, packed, absmax_q, absmax_scales, K: int, blocksize: int = 64,
+                          quant_type="nf4", group: int = 256, out=None, stream=None):
+    """gemm_4bit_backward with the absmax given as double_quant's (codes, scales)."""
+    torch = _torch()
+    _need_cuda(dY, packed, absmax_q, absmax_scales)
+    M, N = dY.shape
+    dX = out if out is not None else torch.empty(M, K, dtype=dY.dtype, device=dY.device)
+    _check(bnb4_gemm_backward_dq(_ptr(dY), _ptr(packed), _ptr(absmax_q), _ptr(absmax_scales), group, _ptr(dX),
+                                 M, N, K, blocksize, _qtype(quant_type), _dtype_code(dY), _stream(stream)),
+           "bnb4_gemm_backward_dq")
     return dX
 
 

@@ -159,8 +159,10 @@ bnb4_status bnb4_gemm(const void *X, const uint8_t *W, const float *absmax, cons
         return from_cuda(launch_gemv(X, W, absmax, nullptr, nullptr, 0, bias, Y, N, K, blocksize, qt, dt, stream));
     // small M: one pass over the weight stream, tensor-core tiles fed from registers
     if (M <= kSmallMMax)
-        return from_cuda(launch_gemm_small(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, stream));
-    return from_cuda(launch_gemm_tc(X, W, absmax, bias, Y, M, N, K, blocksize, qt, dt, false, stream));
+        return from_cuda(launch_gemm_small(X, W, absmax, nullptr, nullptr, 0, bias, Y, M, N, K, blocksize, qt, dt,
+                                           stream));
+    return from_cuda(launch_gemm_tc(X, W, absmax, nullptr, nullptr, 0, bias, Y, M, N, K, blocksize, qt, dt, false,
+                                    stream));
 }
 
 bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *absmax, void *dX,
@@ -172,7 +174,41 @@ bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *W, const float *ab
         return from_cuda(launch_gemm_f32(static_cast<const float *>(dY), W, absmax, nullptr, static_cast<float *>(dX),
                                          M, N, K, blocksize, qt, true, stream));
     if (N % 8 != 0) return BNB4_ERR_SHAPE;  // dY rows are TMA-loaded: 16-byte row pitch
-    return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, dX, M, N, K, blocksize, qt, dt, true, stream));
+    return from_cuda(launch_gemm_tc(dY, W, absmax, nullptr, nullptr, 0, nullptr, dX, M, N, K, blocksize, qt, dt,
+                                    true, stream));
+}
+
+bnb4_status bnb4_gemm_dq(const void *X, const uint8_t *W, const uint8_t *absmax_q, const float *absmax_scales,
+                         int group, const void *bias, void *Y, int64_t M, int64_t N, int64_t K, int blocksize,
+                         bnb4_quant_type qt, bnb4_dtype dt, cudaStream_t stream) {
+    if (!absmax_scales) return BNB4_ERR_NULL;
+    if (!aligned16(absmax_scales)) return BNB4_ERR_ALIGN;
+    bnb4_status s = check_matmul(X, W, reinterpret_cast<const float *>(absmax_q), bias, Y, M, N, K, blocksize, qt,
+                                 dt, false);
+    if (s != BNB4_OK) return s;
+    if (group < 32 || group > 4096 || (group & (group - 1)) != 0) return BNB4_ERR_BLOCKSIZE;
+    if (M == 1 && N <= gemv_max_rows() && K <= gemv_max_k())
+        return from_cuda(launch_gemv(X, W, nullptr, absmax_q, absmax_scales, group, bias, Y, N, K, blocksize, qt,
+                                     dt, stream));
+    if (M <= kSmallMMax)
+        return from_cuda(launch_gemm_small(X, W, nullptr, absmax_q, absmax_scales, group, bias, Y, M, N, K,
+                                           blocksize, qt, dt, stream));
+    return from_cuda(launch_gemm_tc(X, W, nullptr, absmax_q, absmax_scales, group, bias, Y, M, N, K, blocksize,
+                                    qt, dt, false, stream));
+}
+
+bnb4_status bnb4_gemm_backward_dq(const void *dY, const uint8_t *W, const uint8_t *absmax_q,
+                                  const float *absmax_scales, int group, void *dX, int64_t M, int64_t N, int64_t K,
+                                  int blocksize, bnb4_quant_type qt, bnb4_dtype dt, cudaStream_t stream) {
+    if (!absmax_scales) return BNB4_ERR_NULL;
+    if (!aligned16(absmax_scales)) return BNB4_ERR_ALIGN;
+    bnb4_status s = check_matmul(dY, W, reinterpret_cast<const float *>(absmax_q), nullptr, dX, M, N, K, blocksize,
+                                 qt, dt, false);
+    if (s != BNB4_OK) return s;
+    if (group < 32 || group > 4096 || (group & (group - 1)) != 0) return BNB4_ERR_BLOCKSIZE;
+    if (N % 8 != 0) return BNB4_ERR_SHAPE;
+    return from_cuda(launch_gemm_tc(dY, W, nullptr, absmax_q, absmax_scales, group, nullptr, dX, M, N, K,
+                                    blocksize, qt, dt, true, stream));
 }
 
 bnb4_status bnb4_double_quant(const float *absmax, int64_t n, int group, uint8_t *absmax_q,

@@ -228,4 +228,24 @@ __device__ __forceinline__ float div255_rn(float s) {
     return __fdiv_rn(s, 255.0f);
 }
 
+// The absmax value at flat index i of a double-quantized absmax array: 8-bit
+// code q[i] times the step RN(scale / 255) of its group, in one correctly
+// rounded fp32 product (the value bnb4_dequant_absmax writes).
+__device__ __forceinline__ float dq_absmax(const uint8_t *__restrict__ q, const float *__restrict__ scales,
+                                           int log2G, int64_t i) {
+    return __fmul_rn((float)__ldg(q + i), div255_rn(__ldg(scales + (i >> log2G))));
+}
+
+// One absmax value of a weight: fp32, or rebuilt from 8-bit statistics when
+// q is given.
+struct AbsmaxSrc {
+    const float *f32;
+    const uint8_t *q;
+    const float *scales;
+    int log2G;
+    __device__ __forceinline__ float operator()(int64_t i) const {
+        return q ? dq_absmax(q, scales, log2G, i) : __ldg(f32 + i);
+    }
+};
+
 }  // namespace bnb4

@@ -110,7 +110,7 @@ __device__ __forceinline__ uint32_t lut_off(uint32_t w, int j) {
 template <typename D, int NT>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_amx,
-                  const __grid_constant__ CUtensorMap tmap_x, const float *__restrict__ absmax,
+                  const __grid_constant__ CUtensorMap tmap_x, const AbsmaxSrc absmax,
                   const uint16_t *__restrict__ bias, uint16_t *__restrict__ Y, int M, int N, int K,
                   int log2B, int amx_tma, int rbox, const __grid_constant__ CodeTable tab) {
     extern __shared__ uint8_t smem_raw[];
@@ -171,11 +171,11 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_const
             if (!__all_sync(FULL, ok)) break;
             const int b = b_lo + q * RPS;                  // first run of the stage
             const int x0 = ((b * RUN) >> log2B) & ~3;      // first scale of the absmax box
-            if (!amx_tma)  // absmax rows not 16-byte pitched: gather the stage's scales
+            if (!amx_tma)  // absmax rows not 16-byte pitched, or 8-bit statistics: gather the stage's scales
                 for (int p = lane; p < R; p += 32)
                     for (int j = 0; j < RPS && b + j < b_hi; ++j) {
                         const int blk = ((b + j) * RUN) >> log2B;
-                        s.amx[st][p * 4 + (blk - x0)] = __ldg(absmax + (int64_t)(r0 + p) * nblk + blk);
+                        s.amx[st][p * 4 + (blk - x0)] = absmax((int64_t)(r0 + p) * nblk + blk);
                     }
             __syncwarp();  // the gathered scales are written before lane 0 arrives
             if (lane == 0) {
@@ -379,7 +379,7 @@ Plan make_plan(int N, int nb) {
 }
 
 template <typename D, int NT>
-cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const void *bias, void *Y,
+cudaError_t launch_t(const void *X, const uint8_t *W, const AbsmaxSrc &absmax, const void *bias, void *Y,
                      int M, int N, int K, int log2B, const CodeTable &tab, cudaStream_t stream) {
     if (!get_encode()) return cudaErrorNotSupported;
     const int nb = K / RUN;
@@ -393,10 +393,12 @@ cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const
                   CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
         encode_2d(&map_x, xt, X, K, M, (uint64_t)K * 2, RUN, NTOK, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    // absmax by 16-byte TMA boxes when its row pitch allows, else (or for
+    // 8-bit statistics) gathered by the producer warp
     const int nblk = K >> log2B;
-    int amx_tma = nblk % 4 == 0 ? 1 : 0;
+    int amx_tma = (nblk % 4 == 0 && !absmax.q) ? 1 : 0;
     std::memset(&map_amx, 0, sizeof(map_amx));
-    if (amx_tma && encode_2d(&map_amx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, absmax, nblk, N, (uint64_t)nblk * 4, 4,
+    if (amx_tma && encode_2d(&map_amx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, absmax.f32, nblk, N, (uint64_t)nblk * 4, 4,
                              rbox, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
         amx_tma = 0;
     cudaError_t e = set_smem_attr<D, NT>();
@@ -412,13 +414,14 @@ cudaError_t launch_t(const void *X, const uint8_t *W, const float *absmax, const
 
 cudaError_t gemm_small_timeouts_address(unsigned int **p) { return wait_timeouts_address(p); }
 
-cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
-                              const void *bias, void *Y, int64_t M, int64_t N, int64_t K,
-                              int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax_f32, const uint8_t *absmax_q,
+                              const float *scales, int group, const void *bias, void *Y, int64_t M, int64_t N,
+                              int64_t K, int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
                               cudaStream_t stream) {
     static const CodeTable nf4 = host_code_table(BNB4_NF4);
     static const CodeTable fp4 = host_code_table(BNB4_FP4);
     const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
+    const AbsmaxSrc absmax{absmax_f32, absmax_q, scales, absmax_q ? ilog2(group) : 0};
     const int log2B = ilog2(blocksize);
     const int m = (int)M, n = (int)N, k = (int)K;
     if (dt == BNB4_F16) {

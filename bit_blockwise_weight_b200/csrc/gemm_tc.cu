@@ -119,7 +119,7 @@ __device__ __forceinline__ void store_out(uint16_t *out, int64_t row, int n_out,
 template <typename D, bool BWD, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_w,
-               const __grid_constant__ CUtensorMap tmap_amx, const float *__restrict__ absmax,
+               const __grid_constant__ CUtensorMap tmap_amx, const AbsmaxSrc absmax,
                const uint16_t *__restrict__ bias, uint16_t *__restrict__ out, int M, int N, int K,
                int log2B, int amx_tma, const __grid_constant__ CodeTable tab) {
     extern __shared__ uint8_t smem_raw[];
@@ -218,12 +218,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                         blk = (c0 + 64 * (p >> 6)) >> log2B;
                         idx = blk - bwd_x0;
                         if (p < 64 * 4) dst[(p & 63) * 4 + idx] =
-                            (row < N && blk < nblk) ? __ldg(absmax + (int64_t)row * nblk + blk) : 0.0f;
+                            (row < N && blk < nblk) ? absmax((int64_t)row * nblk + blk) : 0.0f;
                     } else {
                         row = c0 + p;
                         blk = (it * BK) >> log2B;
                         idx = blk & 3;
-                        if (p < BN) dst[p * 4 + idx] = row < N ? __ldg(absmax + (int64_t)row * nblk + blk) : 0.0f;
+                        if (p < BN) dst[p * 4 + idx] = row < N ? absmax((int64_t)row * nblk + blk) : 0.0f;
                     }
                 }
             }
@@ -500,7 +500,7 @@ int cluster_capacity(int C) {
 
 template <typename D, bool BWD, int BN>
 cudaError_t launch_bn(const CUtensorMap &map_a, const CUtensorMap &map_w, const CUtensorMap &map_amx,
-                      const float *absmax, const void *bias, void *out, int M, int N, int K,
+                      const AbsmaxSrc &absmax, const void *bias, void *out, int M, int N, int K,
                       int log2B, int amx_tma, const CodeTable &tab, int C, cudaStream_t stream) {
     cudaError_t e = set_smem_attr<D, BWD, BN>();
     if (e != cudaSuccess) return e;
@@ -543,7 +543,7 @@ Plan make_plan(long mt, int n_out, int iters) {
 }
 
 template <typename D, bool BWD>
-cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const void *bias,
+cudaError_t launch_t(const void *A, const uint8_t *W, const AbsmaxSrc &absmax, const void *bias,
                      void *out, int M, int N, int K, int log2B, const CodeTable &tab,
                      cudaStream_t stream) {
     if (!get_encode()) return cudaErrorNotSupported;
@@ -572,12 +572,13 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const float *absmax, const
                         CU_TENSOR_MAP_SWIZZLE_32B);
     if (rw != CUDA_SUCCESS) return cudaErrorInvalidValue;
     // absmax [N rows, K / blocksize]: 16-byte boxes when its row pitch allows,
-    // otherwise gathered by the producer warp
+    // otherwise (or when it arrives as 8-bit statistics) gathered by the
+    // producer warp
     const int nblk = K >> log2B;
-    int amx_tma = (nblk % 4 == 0) ? 1 : 0;
+    int amx_tma = (nblk % 4 == 0 && !absmax.q) ? 1 : 0;
     memset(&map_amx, 0, sizeof(map_amx));
     if (amx_tma &&
-        encode_2d(&map_amx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, absmax, nblk, N, (uint64_t)nblk * 4, 4,
+        encode_2d(&map_amx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, absmax.f32, nblk, N, (uint64_t)nblk * 4, 4,
                   BWD ? BK : bn, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
         amx_tma = 0;
 
@@ -613,12 +614,14 @@ cudaError_t launch_selftest_wait_timeout(cudaStream_t stream) {
 
 cudaError_t gemm_tc_timeouts_address(unsigned int **p) { return wait_timeouts_address(p); }
 
-cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax, const void *bias,
+cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax_f32, const uint8_t *absmax_q,
+                           const float *scales, int group, const void *bias,
                            void *D, int64_t M, int64_t N, int64_t K, int blocksize,
                            bnb4_quant_type qt, bnb4_dtype dt, bool backward, cudaStream_t stream) {
     static const CodeTable nf4 = host_code_table(BNB4_NF4);
     static const CodeTable fp4 = host_code_table(BNB4_FP4);
     const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
+    const AbsmaxSrc absmax{absmax_f32, absmax_q, scales, absmax_q ? ilog2(group) : 0};
     const int log2B = ilog2(blocksize);
     const int m = (int)M, n = (int)N, k = (int)K;
     if (dt == BNB4_F16)

@@ -31,17 +31,20 @@ cudaError_t launch_gemv(const void *x, const uint8_t *W, const float *absmax, co
                         cudaStream_t stream);
 
 // 1 <= M <= 16: TMA-staged weights decoded in registers, mma.sync with the
-// 16-row token tile
-cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax,
-                              const void *bias, void *Y, int64_t M, int64_t N, int64_t K,
-                              int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
+// 16-row token tile.  absmax_q == nullptr: fp32 absmax; else 8-bit
+// double-quantized absmax codes with one fp32 scale per `group` codes
+// (absmax_f32 unused)
+cudaError_t launch_gemm_small(const void *X, const uint8_t *W, const float *absmax_f32, const uint8_t *absmax_q,
+                              const float *scales, int group, const void *bias, void *Y, int64_t M, int64_t N,
+                              int64_t K, int blocksize, bnb4_quant_type qt, bnb4_dtype dt,
                               cudaStream_t stream);
 
 // large M: tcgen05 with weight tiles dequantized into shared memory.
 // backward == true computes dX[M, K] = dY[M, N] @ dequant(W) instead.
-cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax,
-                           const void *bias, void *D, int64_t M, int64_t N, int64_t K,
-                           int blocksize, bnb4_quant_type qt, bnb4_dtype dt, bool backward,
+// (absmax as for launch_gemm_small)
+cudaError_t launch_gemm_tc(const void *A, const uint8_t *W, const float *absmax_f32, const uint8_t *absmax_q,
+                           const float *scales, int group, const void *bias, void *D, int64_t M, int64_t N,
+                           int64_t K, int blocksize, bnb4_quant_type qt, bnb4_dtype dt, bool backward,
                            cudaStream_t stream);
 
 // fp32 compute dtype (x, bias, y in float32; the exact fp32 dequantized

@@ -21,8 +21,9 @@
  *   bnb4_double_quant,  "mps-bitsandbytes 0.4.7", Functional API, Double
  *   bnb4_dequant_absmax Quantization (double_quant(absmax,
  *                       double_quant_block=256), dequant_absmax).
- *   bnb4_gemv_dq        gemv_4bit whose weight carries the double-quantized
- *                       absmax of the same section (8-bit statistics).
+ *   bnb4_gemv_dq,       gemv_4bit, gemm_4bit and its backward whose weight
+ *   bnb4_gemm_dq,       carries the double-quantized absmax of the same
+ *   bnb4_gemm_backward_dq section (8-bit statistics).
  *   bnb4_quantize_8bit, "Feat/mps gemm 4bit bf16", What runs natively now
  *   bnb4_dequantize_8bit (quantize_blockwise / dequantize_blockwise) and
  *                       Correctness (exact nearest code, no lookup-table snap).
@@ -50,6 +51,11 @@
  *     the code (2^-9 relative in bf16, 2^-12 in fp16).  Either way the result
  *     stays within 5e-3 relative L2 of the float64 product with the
  *     dequantized weights.
+ *   - fp32 compute dtype (bnb4_gemv, bnb4_gemm, bnb4_gemm_backward with dt =
+ *     BNB4_F32): x, bias and y in float32; the weight is the exact fp32
+ *     dequantized value RN32(code * absmax); products and sums are fp32
+ *     FMAs, so the result differs from the float64 product only by fp32
+ *     summation rounding.
  *
  * Weight layout for the matmuls: W is [N, K] row-major (out x in, like a
  * Linear layer's weight) and was quantized as one flat array of N*K
@@ -139,7 +145,7 @@ bnb4_status bnb4_dequantize(const uint8_t *packed, const float *absmax,
  * Matrix-vector product for decode (M == 1): y = x @ dequant(W)^T (+ bias).
  *   x        [K] of dt;  packedW [N, K/2];  absmax [N, K/blocksize];
  *   bias     [N] of dt or NULL;  y [N] of dt (out).
- *   dt in {f16, bf16}; K % blocksize == 0 and K % 32 == 0; N, K >= 1.
+ *   dt in {f32, f16, bf16}; K % blocksize == 0 and K % 32 == 0; N, K >= 1.
  */
 bnb4_status bnb4_gemv(const void *x, const uint8_t *packedW,
                       const float *absmax, const void *bias, void *y,
@@ -191,6 +197,31 @@ bnb4_status bnb4_gemm_backward(const void *dY, const uint8_t *packedW,
                                int64_t N, int64_t K, int blocksize,
                                bnb4_quant_type quant_type, bnb4_dtype dt,
                                cudaStream_t stream);
+
+/*
+ * bnb4_gemm and bnb4_gemm_backward with the weight's absmax given as 8-bit
+ * statistics (see bnb4_double_quant / bnb4_gemv_dq): absmax_q
+ * [N*K/blocksize] codes and absmax_scales [ceil(N*K/blocksize / group)]
+ * fp32, both device pointers, 16-byte aligned.  Each block's absmax is
+ * rebuilt inside the kernel as bnb4_dequant_absmax computes it, so the
+ * result is bit-identical to bnb4_gemm / bnb4_gemm_backward given the
+ * array bnb4_dequant_absmax writes, with no such array in memory.
+ *   dt in {f16, bf16}; group a power of two in [32, 4096]
+ *   (BNB4_ERR_BLOCKSIZE otherwise); other arguments and constraints as for
+ *   bnb4_gemm / bnb4_gemm_backward.
+ */
+bnb4_status bnb4_gemm_dq(const void *X, const uint8_t *packedW,
+                         const uint8_t *absmax_q, const float *absmax_scales,
+                         int group, const void *bias, void *Y, int64_t M,
+                         int64_t N, int64_t K, int blocksize,
+                         bnb4_quant_type quant_type, bnb4_dtype dt,
+                         cudaStream_t stream);
+bnb4_status bnb4_gemm_backward_dq(const void *dY, const uint8_t *packedW,
+                                  const uint8_t *absmax_q,
+                                  const float *absmax_scales, int group,
+                                  void *dX, int64_t M, int64_t N, int64_t K,
+                                  int blocksize, bnb4_quant_type quant_type,
+                                  bnb4_dtype dt, cudaStream_t stream);
 
 /*
  * Double quantization of an absmax array (the pages give the call and the

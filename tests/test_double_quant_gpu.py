@@ -183,3 +183,74 @@ def test_dequant_absmax_every_significand():
         want = oracle.dequant_absmax(q, sc, G)
         for o in range(3):
             assert _same_bits(got[o::G], want[o::G]), o
+
+
+# ------------------------------------------- matmuls with M >= 2 on 8-bit statistics
+
+def _dq_weight(N, K, B, q, group, seed):
+    w = synthetic.weight(N, K, seed, 0.02).numpy().reshape(-1)
+    packed, absmax = oracle.quantize(w, "f32", B, q)
+    dp, da = torch.from_numpy(packed).cuda(), torch.from_numpy(absmax).cuda()
+    aq, asc = bnb4.double_quant(da, group)
+    back = bnb4.dequant_absmax(aq, asc, group)   # the absmax the 8-bit statistics stand for
+    return packed, dp, aq, asc, back
+
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N,K,B,group", [(2, 96, 2048, 64, 256), (9, 45, 1600, 64, 32),
+                                           (16, 64, 4096, 256, 256), (17, 256, 512, 64, 256),
+                                           (300, 264, 704, 64, 64), (300, 96, 256, 128, 1024)])
+def test_gemm_dq_bit_identical_to_fp32_absmax(q, dt, M, N, K, B, group):
+    """gemm_4bit_dq equals gemm_4bit given the absmax dequant_absmax writes, bit
+    for bit (small-M and tcgen05 kernels; absmax rows with and without a 16-byte
+    pitch), and stays within the matmul bar of the float64 oracle."""
+    from gpu_util import MATMUL_TOL, as_f64, rel_l2, to_dev
+    packed, dp, aq, asc, back = _dq_weight(N, K, B, q, group, seed=M + N)
+    Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
+    X = to_dev(Xs, dt).view(M, K)
+    bias = to_dev(synthetic.storage_numpy(synthetic.bias(N, seed=2, dtype=dt)), dt) if M % 2 else None
+    Ydq = to_host(bnb4.gemm_4bit_dq(X, dp, aq, asc, N, bias, B, q, group))
+    Yref = to_host(bnb4.gemm_4bit(X, dp, back, N, bias, B, q))
+    assert np.array_equal(Ydq, Yref)
+    bs = None if bias is None else to_host(bias)
+    ref = oracle.matmul(Xs, dt, packed, to_host(back), bs, M, N, K, B, q)
+    assert rel_l2(as_f64(Ydq, dt).reshape(M, N), ref) <= MATMUL_TOL
+
+
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+@pytest.mark.parametrize("M,N,K,B,group", [(64, 264, 2048, 128, 256), (130, 520, 768, 64, 32)])
+def test_gemm_backward_dq_bit_identical_to_fp32_absmax(q, M, N, K, B, group):
+    from gpu_util import MATMUL_TOL, as_f64, rel_l2, to_dev
+    packed, dp, aq, asc, back = _dq_weight(N, K, B, q, group, seed=N)
+    dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3)).reshape(-1)
+    dY = to_dev(dYs, "bf16").view(M, N)
+    got = to_host(bnb4.gemm_4bit_backward_dq(dY, dp, aq, asc, K, B, q, group))
+    assert np.array_equal(got, to_host(bnb4.gemm_4bit_backward(dY, dp, back, K, B, q)))
+    ref = oracle.matmul_backward(dYs, "bf16", packed, to_host(back), M, N, K, B, q)
+    assert rel_l2(as_f64(got, "bf16").reshape(M, K), ref) <= MATMUL_TOL
+
+
+@pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
+def test_gemm_dq_70b_shapes_m16_sampled(K, N):
+    """M = 16 on the 70B-shaped weights with 8-bit statistics: bit-identical to
+    the fp32-absmax kernel on the inverse's absmax (whole output)."""
+    from gpu_util import to_dev
+    w = synthetic.normal((N * K,), 0, 0.015, "f32", device="cuda")
+    dp, da = bnb4.quantize_4bit(w, 64, "nf4")
+    del w
+    aq, asc = bnb4.double_quant(da, 256)
+    back = bnb4.dequant_absmax(aq, asc, 256)
+    X = synthetic.normal((16, K), 1, 1.0, "bf16", device="cuda")
+    assert torch.equal(bnb4.gemm_4bit_dq(X, dp, aq, asc, N), bnb4.gemm_4bit(X, dp, back, N))
+
+
+def test_gemm_dq_argument_checks():
+    A = 1 << 20
+    g = bnb4.bnb4_gemm_dq
+    assert g(A, A, A, None, 256, None, A, 4, 64, 128, 64, 0, 2, None) == 1       # no scales
+    assert g(A, A, A, A + 4, 256, None, A, 4, 64, 128, 64, 0, 2, None) == 2      # misaligned scales
+    assert g(A, A, A, A, 100, None, A, 4, 64, 128, 64, 0, 2, None) == 3          # group not a power of two
+    assert g(A, A, A, A, 256, None, A, 4, 64, 128, 64, 0, 0, None) == 5          # f32
+    b = bnb4.bnb4_gemm_backward_dq
+    assert b(A, A, A, A, 256, A, 4, 100, 128, 64, 0, 2, None) == 4               # N % 8

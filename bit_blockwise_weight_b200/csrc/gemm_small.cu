@@ -26,7 +26,7 @@
 // X.  The reduction over k is a plain sum, so the order is free, and every
 // step stays inside one run, hence one block.  So the weight a token meets is
 // RN_dtype(code) * absmax, accumulated in fp32; the codes, as 16-bit values,
-// lose at most 2^-9 (bf16) or 2^-12 (f16) relative.
+// lose at most 2^-8 (bf16) or 2^-11 (f16) relative.
 //
 // Work split: CTA (g, z) owns rows [N g / G, N (g+1) / G) (balanced to one
 // row, at most 256) and the z-th of S shares of the K stages; the S CTAs of a

@@ -38,7 +38,7 @@
 // one prmt builds the lane's address (table page, byte, lane) from the packed
 // word and the lookup never conflicts.  The codes enter as 16-bit values (the
 // code table rounded once to bf16 / fp16), so the weight a product meets is
-// RN_dtype(code) * absmax: 2^-9 (bf16) or 2^-12 (fp16) relative to the
+// RN_dtype(code) * absmax: 2^-8 (bf16) or 2^-11 (fp16) relative to the
 // dequantized value.
 //
 // Work split: CTA c owns rows [N c / G, N (c+1) / G) (balanced to one row) and

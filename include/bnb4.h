@@ -48,7 +48,7 @@
  *     value above (already in the compute dtype).  For M <= 16 (gemv
  *     included) each code is rounded to the compute dtype and the fp32 sums
  *     are scaled by the block's absmax: the same weight up to one rounding of
- *     the code (2^-9 relative in bf16, 2^-12 in fp16).  Either way the result
+ *     the code (2^-8 relative in bf16, 2^-11 in fp16).  Either way the result
  *     stays within 5e-3 relative L2 of the float64 product with the
  *     dequantized weights.
  *   - fp32 compute dtype (bnb4_gemv, bnb4_gemm, bnb4_gemm_backward with dt =

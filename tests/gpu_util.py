@@ -42,3 +42,28 @@ def unpack_nibbles(packed: np.ndarray, n: int) -> np.ndarray:
     out[0::2] = p >> 4
     out[1::2] = p & 15
     return out[:n]
+
+
+# Unit roundoff of the 16-bit compute dtypes: bf16 has an 8-bit significand,
+# fp16 an 11-bit one, so rounding to them moves a value by at most 2^-8 / 2^-11
+# of itself.
+UNIT_ROUNDOFF = {"bf16": 2.0 ** -8, "f16": 2.0 ** -11}
+
+
+def elementwise_excess(got, ref, absdot, dt, K):
+    """How far the worst output lies outside its own error bound (<= 0: every
+    output inside).  The 16-bit matmuls meet the weight rounded once to the
+    compute dtype (RN_dt(code) * absmax, or RN_dt(code * absmax)), multiply it
+    exactly by x in fp32, sum in fp32 and round the result once to the dtype:
+        |y - y_ref| <= u_dt (sum_k |x_k w_k| + |b|) + u_dt |y_ref|
+                       + (K + 4) 2^-24 (sum_k |x_k w_k| + |b|)
+    with a 1 % margin and an absolute floor at the smallest fp16 subnormal.
+    absdot is sum_k |x_k w_k| + |b| per output.  A localised mistake (one
+    block's scale, one column) breaks this bound long before it moves the
+    relative L2 over the whole tensor."""
+    u = UNIT_ROUNDOFF[dt]
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    absdot = np.asarray(absdot, np.float64)
+    tol = 1.01 * (u * absdot + u * np.abs(ref)) + (K + 4) * 2.0 ** -24 * absdot + 2.0 ** -24
+    return float(np.max(np.abs(got - ref) - tol))

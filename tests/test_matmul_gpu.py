@@ -11,7 +11,7 @@ import bit_blockwise_weight_b200 as bnb4
 import oracle
 import synthetic
 
-from gpu_util import MATMUL_TOL, as_f64, rel_l2, to_dev, to_host
+from gpu_util import MATMUL_TOL, as_f64, elementwise_excess, rel_l2, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
 
@@ -25,6 +25,32 @@ class Weight:
         self.packed, self.absmax = oracle.quantize(w, "f32", B, q)
         self.dp = torch.from_numpy(self.packed).cuda()
         self.da = torch.from_numpy(self.absmax).cuda()
+        self._absw = None
+
+    def absw(self):
+        """|dequantized fp32 weight| [N, K] in float64 (for the per-element bounds)."""
+        if self._absw is None:
+            w = oracle.dequantize(self.packed, self.absmax, self.N * self.K, self.B, self.q, "f32")
+            self._absw = np.abs(w.astype(np.float64)).reshape(self.N, self.K)
+        return self._absw
+
+    def absw_rows(self, rows):
+        """|dequantized fp32 weight| of the given rows only, [len(rows), K] float64."""
+        hb, nb = self.K // 2, self.K // self.B
+        p = np.concatenate([self.packed[r * hb:(r + 1) * hb] for r in rows])
+        a = np.concatenate([self.absmax[r * nb:(r + 1) * nb] for r in rows])
+        w = oracle.dequantize(p, a, len(rows) * self.K, self.B, self.q, "f32")
+        return np.abs(w.astype(np.float64)).reshape(len(rows), self.K)
+
+
+def _absdot(Xs, dt, absw_rows, bias_s=None):
+    """sum_k |x_mk w_jk| (+ |b_j|) for every (m, j) of X [M, K] and the given weight rows."""
+    K = absw_rows.shape[1]
+    ax = np.abs(as_f64(Xs, dt)).reshape(-1, K)
+    d = ax @ absw_rows.T
+    if bias_s is not None:
+        d = d + np.abs(as_f64(bias_s, dt))[None, :]
+    return d
 
 
 def _ref_forward(Wt, Xs, dt, bias_s, rows=None):
@@ -53,8 +79,10 @@ def test_gemv_small_shapes(q, dt, N, K, B, with_bias):
     y = bnb4.gemv_4bit(to_dev(xs, dt), Wt.dp, Wt.da, N, K, None if bs is None else to_dev(bs, dt),
                        B, q)
     ref = _ref_forward(Wt, xs, dt, bs)[0]
-    err = rel_l2(as_f64(to_host(y), dt), ref)
+    got = as_f64(to_host(y), dt)
+    err = rel_l2(got, ref)
     assert err <= MATMUL_TOL, err
+    assert elementwise_excess(got, ref, _absdot(xs, dt, Wt.absw(), bs)[0], dt, K) <= 0
 
 
 @pytest.mark.parametrize("K,N", [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)])
@@ -68,8 +96,11 @@ def test_gemv_llama_decode_shapes_sampled(K, N, with_bias):
                                None if bs is None else to_dev(bs, "bf16"), 64, "nf4"))
     rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(K + N).integers(0, N, 254)]))
     ref = _ref_forward(Wt, xs, "bf16", bs, rows)[0]
-    err = rel_l2(as_f64(y, "bf16")[rows], ref)
+    got = as_f64(y, "bf16")[rows]
+    err = rel_l2(got, ref)
     assert err <= MATMUL_TOL, err
+    ad = _absdot(xs, "bf16", Wt.absw_rows(rows))[0] + (0 if bs is None else np.abs(as_f64(bs, "bf16"))[rows])
+    assert elementwise_excess(got, ref, ad, "bf16", K) <= 0
 
 
 # -------------------------------------------------------------- small-M gemm
@@ -86,8 +117,10 @@ def test_gemm_small_m(q, dt, M, N, K, B):
     Y = bnb4.gemm_4bit(to_dev(Xs, dt).view(M, K), Wt.dp, Wt.da, N,
                        None if bs is None else to_dev(bs, dt), B, q)
     ref = _ref_forward(Wt, Xs, dt, bs)
-    err = rel_l2(as_f64(to_host(Y), dt).reshape(M, N), ref)
+    got = as_f64(to_host(Y), dt).reshape(M, N)
+    err = rel_l2(got, ref)
     assert err <= MATMUL_TOL, err
+    assert elementwise_excess(got, ref, _absdot(Xs, dt, Wt.absw(), bs), dt, K) <= 0
 
 
 @pytest.mark.parametrize("q", ["nf4", "fp4"])
@@ -97,12 +130,15 @@ def test_gemm_small_m_70b_shapes_sampled(q, dt, K, N):
     """70B-shaped projections, M in {1,2,4,8,16}, sigma 0.015: sampled rows."""
     Wt = Weight(N, K, 64, q, seed=0, sigma=0.015)
     rows = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(K).integers(0, N, 62)]))
+    absw_r = Wt.absw_rows(rows)
     for M in (1, 2, 4, 8, 16):
         Xs = synthetic.storage_numpy(synthetic.activations(M, K, seed=1, dtype=dt)).reshape(-1)
         Y = to_host(bnb4.gemm_4bit(to_dev(Xs, dt).view(M, K), Wt.dp, Wt.da, N, None, 64, q))
         ref = _ref_forward(Wt, Xs, dt, None, rows)
-        err = rel_l2(as_f64(Y, dt).reshape(M, N)[:, rows], ref)
+        got = as_f64(Y, dt).reshape(M, N)[:, rows]
+        err = rel_l2(got, ref)
         assert err <= MATMUL_TOL, (M, err)
+        assert elementwise_excess(got, ref, _absdot(Xs, dt, absw_r), dt, K) <= 0, M
 
 
 # ---------------------------------------------- large-M gemm and backward (tcgen05)
@@ -131,8 +167,10 @@ def test_gemm_large_m(q, dt, M, N, K, B):
     Y = bnb4.gemm_4bit(to_dev(Xs, dt).view(M, K), Wt.dp, Wt.da, N,
                        None if bs is None else to_dev(bs, dt), B, q)
     ref = _ref_forward(Wt, Xs, dt, bs)
-    err = rel_l2(as_f64(to_host(Y), dt).reshape(M, N), ref)
+    got = as_f64(to_host(Y), dt).reshape(M, N)
+    err = rel_l2(got, ref)
     assert err <= MATMUL_TOL, err
+    assert elementwise_excess(got, ref, _absdot(Xs, dt, Wt.absw(), bs), dt, K) <= 0
 
 
 @pytest.mark.parametrize("q", ["nf4", "fp4"])
@@ -150,8 +188,11 @@ def test_gemm_backward(q, dt, M, N, K, B):
     dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3, dtype=dt)).reshape(-1)
     dX = bnb4.gemm_4bit_backward(to_dev(dYs, dt).view(M, N), Wt.dp, Wt.da, K, B, q)
     ref = _ref_backward(Wt, dYs, dt, M)
-    err = rel_l2(as_f64(to_host(dX), dt).reshape(M, K), ref)
+    got = as_f64(to_host(dX), dt).reshape(M, K)
+    err = rel_l2(got, ref)
     assert err <= MATMUL_TOL, err
+    ad = np.abs(as_f64(dYs, dt)).reshape(M, N) @ Wt.absw()
+    assert elementwise_excess(got, ref, ad, dt, N) <= 0
 
 
 @pytest.mark.parametrize("M", [512, 2048])
@@ -168,6 +209,9 @@ def test_prefill_and_backward_full_size_sampled(M):
     ref = oracle.matmul_entries(Xs, "bf16", Wt.packed, Wt.absmax, None, M, N, K, 64, "nf4", ms, js)
     err = rel_l2(Y[ms, js], ref)
     assert err <= MATMUL_TOL, ("forward", err)
+    ax = np.abs(as_f64(Xs, "bf16")).reshape(M, K)
+    aw = Wt.absw()
+    assert elementwise_excess(Y[ms, js], ref, (ax[ms] * aw[js]).sum(1), "bf16", K) <= 0, "forward"
     dYs = synthetic.storage_numpy(synthetic.grad_output(M, N, seed=3)).reshape(-1)
     dX = as_f64(to_host(bnb4.gemm_4bit_backward(to_dev(dYs, "bf16").view(M, N), Wt.dp, Wt.da, K)),
                 "bf16").reshape(M, K)
@@ -176,3 +220,5 @@ def test_prefill_and_backward_full_size_sampled(M):
     refb = _ref_backward(Wt, dYs, "bf16", M, (ms2, ks))
     err = rel_l2(dX[ms2, ks], refb)
     assert err <= MATMUL_TOL, ("backward", err)
+    ady = np.abs(as_f64(dYs, "bf16")).reshape(M, N)
+    assert elementwise_excess(dX[ms2, ks], refb, (ady[ms2] * aw[:, ks].T).sum(1), "bf16", N) <= 0, "backward"

@@ -213,3 +213,39 @@ def test_full_size_2p28_sampled_blocks(dtype, seeds):
                 del packed, absmax, deq, p2, a2, a_el, err
         del xd
         torch.cuda.empty_cache()
+
+
+def test_full_size_2p28_every_run_whole_tensor_digests():
+    """Every run of the full-size round-trip sweep (2^28 elements, seeds 0..3,
+    fp32 / fp16 / bf16, NF4 / FP4, blocksizes 64..4096: 168 runs): the SHA-256
+    digests of the GPU's packed bytes, absmax and dequantized tensor equal the
+    CPU oracle's, stored in tests/golden/roundtrip_2p28_digests.json by
+    tests/golden/make_roundtrip_digests.py (which calls only the oracle).  So
+    every element of every run is compared, not a sample."""
+    import hashlib
+    import json
+    import os
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "roundtrip_2p28_digests.json")
+    with open(path) as f:
+        doc = json.load(f)
+    n = doc["n"]
+
+    def digest(t):
+        return hashlib.sha256(memoryview(to_host(t)).cast("B")).hexdigest()
+
+    bad = []
+    torch_dt = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
+    for seed in doc["seeds"]:
+        for dt in doc["dtypes"]:
+            x = synthetic.roundtrip_tensor(n, seed, dt).cuda()
+            deq = torch.empty(n, dtype=torch_dt[dt], device="cuda")
+            for qt in doc["quant_types"]:
+                for B in doc["blocksizes"]:
+                    packed, absmax = bnb4.quantize_4bit(x, B, qt)
+                    bnb4.dequantize_4bit(packed, absmax, n, B, qt, out=deq)
+                    want = doc["runs"][f"{dt}/{qt}/B{B}/seed{seed}"]
+                    got = {"packed": digest(packed), "absmax": digest(absmax), "dequant": digest(deq)}
+                    bad += [(f"{dt}/{qt}/B{B}/seed{seed}", k) for k in got if got[k] != want[k]]
+                    del packed, absmax
+            del x, deq
+    assert len(doc["runs"]) == 168 and not bad, bad[:8]

@@ -32,7 +32,9 @@
  *      bias, with no rounding of the result.
  *   R9 double quantization of absmax (see oracle_double_quant).
  *   R10 8-bit blockwise: steps R3-R5 and R7 with a caller's 256-entry code
- *      table and one code index per byte (see oracle_quantize_8bit).
+ *      table and one code index per byte (see oracle_quantize_8bit); the
+ *      nearest entry is decided on exact distances (a caller's table may
+ *      hold -c and +c, where float64 distances would tie tiny quotients).
  *   R11 4-bit embedding lookup: rows of a table quantized as one flat array
  *      (see oracle_embedding_4bit).
  */
@@ -441,14 +443,41 @@ static int code8_usable(const float *code)
     return 1;
 }
 
+/* |v - c| exactly, as hi + lo with hi = RN(|v - c|) in float64 and lo the
+ * rounding error (Knuth's TwoSum; exact, no underflow for fp32 inputs).  A
+ * plain float64 difference is not exact once |v| is below 2^-53 |c|: with a
+ * table holding -c and +c (a decision threshold of exactly 0) it would call
+ * every tiny v a tie. */
+struct dist2 {
+    double hi, lo;
+};
+static struct dist2 exact_distance(float v, float c)
+{
+    const double a = v, b = -(double)c;
+    const double s = a + b, bb = s - a;
+    const double err = (a - (s - bb)) + (b - bb);
+    struct dist2 d = {s, err};
+    if (s < 0.0) {
+        d.hi = -s;
+        d.lo = -err;
+    }
+    return d;
+}
+/* x < y for exact values hi + lo: hi is the rounded value, so hi decides
+ * unless the two are equal */
+static int dist_less(struct dist2 x, struct dist2 y)
+{
+    return x.hi < y.hi || (x.hi == y.hi && x.lo < y.lo);
+}
+
 /* R10 (as R5): exact nearest of the 256 entries, ties to the smallest index. */
 static int nearest_code8(float v, const float *code)
 {
     int best_j = 0;
-    double best_d = fabs((double)v - (double)code[0]);
+    struct dist2 best_d = exact_distance(v, code[0]);
     for (int j = 1; j < 256; ++j) {
-        const double dist = fabs((double)v - (double)code[j]);
-        if (dist < best_d) {
+        const struct dist2 dist = exact_distance(v, code[j]);
+        if (dist_less(dist, best_d)) {
             best_d = dist;
             best_j = j;
         }

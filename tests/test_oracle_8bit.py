@@ -231,3 +231,35 @@ def test_table_validation():
             oracle.quantize_8bit(x, "f32", 4, t)
         with pytest.raises(ValueError):
             oracle.dequantize_8bit(np.zeros(8, np.uint8), np.ones(2, np.float32), 8, 4, t, "f32")
+
+
+def test_symmetric_pair_decides_tiny_quotients_by_sign():
+    """A table whose two smallest entries are -c and +c has a decision threshold
+    of exactly 0.  A quotient v = x / absmax far below c is nearer +c when
+    positive and -c when negative; a distance taken in float64 (c + |v| and
+    c - |v| both rounding to c) would call every such v a tie.  Checked against
+    the exact rational restatement, with quotients down to the subnormal range."""
+    rng = np.random.default_rng(23)
+    c = np.float32(2.0 ** -24)
+    vals = {-1.0, 1.0, -float(c), float(c)}
+    while len(vals) < 256:
+        v = float(np.float32(rng.uniform(-1.0, 1.0)))
+        if abs(v) >= 2.0 ** -20:
+            vals.add(v)
+    code = np.array(sorted(vals), np.float32)
+    B = 64
+    a = np.float32(1.2680464e-18)
+    tiny = np.concatenate([np.float32(a) * np.exp2(-np.arange(30, 120, 6, dtype=np.float64)).astype(np.float32),
+                           np.array([1.4e-45, 2.8e-45, 1e-40, 1e-30], np.float32)])
+    tiny = tiny[tiny > 0]                          # (the deepest scalings underflow)
+    x = np.zeros(B, np.float32)
+    x[0] = a
+    x[1:1 + tiny.size] = tiny
+    x[1 + tiny.size:1 + 2 * tiny.size] = -tiny
+    x[2 * tiny.size + 1] = -0.0
+    q, _ = oracle.quantize_8bit(x, "f32", B, code)
+    codes = [Fraction(float(v)) for v in code]
+    idxs, _ = bf.quantize_with_table([Fraction(float(v)) for v in x], B, codes)
+    assert list(q) == idxs
+    k = int(np.searchsorted(code, 0.0))            # index of +c
+    assert all(i == k for i in q[1:1 + tiny.size]) and all(i == k - 1 for i in q[1 + tiny.size:1 + 2 * tiny.size])

@@ -54,7 +54,9 @@ MUTATIONS = {
     "quantize_8bit_snaps_to_grid": ("q[i] = (uint8_t)nearest_code8(v, code);",
                                     "q[i] = (uint8_t)nearest_code8((float)(nearbyint(((double)v + 1.0) * 32767.5)"
                                     " / 32767.5 - 1.0), code);"),
-    "quantize_8bit_ties_to_largest": ("if (dist < best_d) {", "if (dist <= best_d) {"),
+    "quantize_8bit_ties_to_largest": ("if (dist_less(dist, best_d)) {", "if (!dist_less(best_d, dist)) {"),
+    "quantize_8bit_float64_distance": ("return x.hi < y.hi || (x.hi == y.hi && x.lo < y.lo);",
+                                       "return x.hi < y.hi;"),
     "quantize_8bit_absmax_without_abs": ("const float mag = fabsf(load_elem(x, dtype, i));",
                                          "const float mag = load_elem(x, dtype, i);"),
     "dequantize_8bit_skips_fp32_rounding": (
@@ -87,6 +89,7 @@ PIN_CHECKS = [
     lambda: q8_pins.test_dyadic_linear_table_closed_form(),
     lambda: [q8_pins.test_every_midpoint_neighbourhood(k) for k in ("uniform", "log")],
     lambda: q8_pins.test_special_blocks(),
+    lambda: q8_pins.test_symmetric_pair_decides_tiny_quotients_by_sign(),
     lambda: q8_pins.test_dequant_double_rounding(),
     lambda: [emb_pins.test_matches_exact_rationals(q, D, B) for q in ("nf4", "fp4") for D, B in ((12, 4), (13, 4))],
     lambda: emb_pins.test_index_checks(),

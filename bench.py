@@ -826,6 +826,7 @@ def run_reference(args):
 PROFILE_CASES = {
     # name: what runs (inputs above L2 size, a few hundred MB on the device at most)
     "quantize": "quantize_4bit, 2^26 bf16 elements, NF4, B=64",
+    "quantize_fp4": "quantize_4bit, 2^26 bf16 elements, FP4, B=64",
     "dequantize": "dequantize_4bit, 2^26 elements to bf16, NF4, B=64",
     "gemv": "gemv_4bit + bias, K=4096, N=14336, NF4 B=64, bf16",
     "gemm_small": "gemm_4bit M=16, K=8192, N=28672, NF4 B=64, bf16",
@@ -847,9 +848,9 @@ def profile_case(name):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     d = str(dev)
-    if name in ("quantize", "dequantize"):
+    if name in ("quantize", "dequantize", "quantize_fp4"):
         x = synthetic.roundtrip_tensor(1 << 26, 0, "bf16", device=d)
-        p, a = bnb4.quantize_4bit(x, BLOCK, "nf4")
+        p, a = bnb4.quantize_4bit(x, BLOCK, "fp4" if name == "quantize_fp4" else "nf4")
         if name == "dequantize":
             bnb4.dequantize_4bit(p, a, x.numel(), BLOCK, "nf4", dtype=torch.bfloat16)
     elif name == "double_quant":

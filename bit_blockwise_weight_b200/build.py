@@ -44,7 +44,7 @@ def build(force: bool = False, verbose: bool = False, extra: list | None = None)
 
     def compile_one(src):
         obj = os.path.join(OBJ, os.path.basename(src) + ".o")
-        cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-dc" if False else "-c", src, "-o", obj]
+        cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)

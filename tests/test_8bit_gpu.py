@@ -110,3 +110,57 @@ def test_full_size_sample():
     assert np.array_equal(to_host(ga), oa) and np.array_equal(to_host(gq), oq)
     gd = to_host(bnb4.dequantize_8bit(gq, ga, code, 64, dtype=torch.bfloat16))
     assert _same16(gd, oracle.dequantize_8bit(oq, oa, n, 64, code, "bf16"))
+
+
+def _straddle_table(symmetric: bool) -> np.ndarray:
+    """Entries spread over [-1, 1] with no 0 and the two smallest magnitudes
+    straddling it: -2^-24 and +2^-24 give a threshold of exactly 0, -2^-24 and
+    the float after 2^-24 one of 2^-48 (the smallest a table can have)."""
+    rng = np.random.default_rng(21)
+    lo = np.float32(2.0 ** -24)
+    hi = lo if symmetric else np.nextafter(lo, np.float32(1))
+    vals = {-1.0, 1.0, -float(lo), float(hi)}
+    while len(vals) < 256:
+        v = float(np.float32(rng.uniform(-1.0, 1.0)))
+        if abs(v) >= 2.0 ** -20:
+            vals.add(v)
+    return np.array(sorted(vals), np.float32)
+
+
+@pytest.mark.parametrize("kind", ["log", "straddle", "symmetric"])
+def test_midpoints_over_the_exponent_range(kind):
+    """Values next to every midpoint times absmax, for absmax over the whole
+    exponent range (around the limits below which the reciprocal path gives
+    way to the division: 2^-96, and the table's own floor), plus elements
+    whose quotients are tiny or subnormal next to thresholds of 0 and 2^-48."""
+    code = _table("log", seed=5) if kind == "log" else _straddle_table(kind == "symmetric")
+    mids = (code[:-1].astype(np.float64) + code[1:].astype(np.float64)) / 2
+    rng = np.random.default_rng(17)
+    exps = np.concatenate([[-126, -120, -100, -97, -96, -95, -80, -60, -54, -53, -52, -51, -30, -1, 0,
+                            40, 95, 96, 97, 126, 127], rng.integers(-126, 128, 27)])
+    a_all = (rng.uniform(1.0, 2.0, exps.size) * np.exp2(exps.astype(np.float64))).astype(np.float32)
+    a_all = a_all[np.isfinite(a_all)]
+    B = 64
+    blocks = []
+    for a in a_all:
+        x0 = (mids * np.float64(a)).astype(np.float32)
+        cand = [x0]
+        up, dn = x0, x0
+        for _ in range(3):
+            up, dn = np.nextafter(up, np.float32(np.inf)), np.nextafter(dn, np.float32(-np.inf))
+            cand += [up, dn]
+        tiny = np.float32(a) * np.exp2(-np.arange(40, 160, 4, dtype=np.float64)).astype(np.float32)
+        c = np.concatenate(cand + [tiny, -tiny])
+        c = c[np.isfinite(c) & (np.abs(c) <= a)]
+        for j in range(0, c.size, B - 1):
+            blk = np.zeros(B, np.float32)
+            blk[0] = a
+            part = c[j:j + B - 1]
+            blk[1:1 + part.size] = part
+            blocks.append(blk)
+    x = np.concatenate(blocks)
+    gq, ga = bnb4.quantize_8bit(torch.from_numpy(x).cuda(), code, B)
+    oq, oa = oracle.quantize_8bit(x, "f32", B, code)
+    assert np.array_equal(to_host(ga).view(np.uint32), oa.view(np.uint32))
+    bad = np.nonzero(to_host(gq) != oq)[0]
+    assert bad.size == 0, (bad.size, x[bad[:4]], x[(bad[:4] // B) * B])

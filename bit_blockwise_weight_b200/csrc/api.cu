@@ -285,16 +285,15 @@ bnb4_status bnb4_device_status(cudaStream_t stream) {
         unsigned int v = 0;
         if (cudaMemcpy(&v, w[i], sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return BNB4_ERR_CUDA;
         if (v == 0) continue;
-        // one atomic exchange on the device: an increment that lands after the
-        // read above is taken with it, never lost
-        take_counter_kernel<<<1, 1, 0, stream>>>(w[i]);
-        if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess) return BNB4_ERR_CUDA;
-        // both timeout words are one status
-        if (i == 1) {
-            take_counter_kernel<<<1, 1, 0, stream>>>(w[2]);
-            if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(stream) != cudaSuccess)
-                return BNB4_ERR_CUDA;
+        // one atomic exchange on the device per word: an increment that lands
+        // after the read above is taken with it, never lost.  The timeout
+        // words (one per kernel file) are one status and are taken together.
+        const int last = code[i] == BNB4_ERR_TIMEOUT ? 2 : i;
+        for (int j = i; j <= last; ++j) {
+            take_counter_kernel<<<1, 1, 0, stream>>>(w[j]);
+            if (cudaGetLastError() != cudaSuccess) return BNB4_ERR_CUDA;
         }
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return BNB4_ERR_CUDA;
         return code[i];
     }
     return BNB4_OK;

@@ -313,9 +313,7 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
     if (ng > 0) load(cq, css, ua);
     {
         // table: entry v (codes of nibbles v >> 4, v & 15) copied to words 64 v + l, l < 32
-#pragma unroll
-        for (int i = 0; i < 2048 / kThreads; ++i) {
-            const int idx = tid + i * kThreads;              // 2048 16-byte pieces
+        for (int idx = tid; idx < 2048; idx += kThreads) {   // 2048 16-byte pieces
             const int v = idx >> 3, q = idx & 7;
             const uint32_t e = Dt<D>::pack2(tab.v[v >> 4], tab.v[v & 15]);
             sts128(lut_a + v * 256 + q * 16, make_uint4(e, e, e, e));

@@ -236,6 +236,14 @@ __device__ __forceinline__ float dq_absmax(const uint8_t *__restrict__ q, const 
     return __fmul_rn((float)__ldg(q + i), div255_rn(__ldg(scales + (i >> log2G))));
 }
 
+// The loads behind one absmax value, before any arithmetic: the fp32 value,
+// or the 8-bit code and its group's scale.  Kernels that fetch a stage ahead
+// hold these in registers, so no use of a load sits next to its issue.
+struct AbsmaxRaw {
+    uint32_t code;
+    float v;  // the fp32 absmax, or the group scale when the source is 8-bit
+};
+
 // One absmax value of a weight: fp32, or rebuilt from 8-bit statistics when
 // q is given.
 struct AbsmaxSrc {
@@ -245,6 +253,14 @@ struct AbsmaxSrc {
     int log2G;
     __device__ __forceinline__ float operator()(int64_t i) const {
         return q ? dq_absmax(q, scales, log2G, i) : __ldg(f32 + i);
+    }
+    __device__ __forceinline__ AbsmaxRaw raw(int64_t i) const {
+        if (q) return AbsmaxRaw{(uint32_t)__ldg(q + i), __ldg(scales + (i >> log2G))};
+        return AbsmaxRaw{0u, __ldg(f32 + i)};
+    }
+    // the same value as operator() on the same index
+    __device__ __forceinline__ float finish(const AbsmaxRaw &r) const {
+        return q ? __fmul_rn((float)r.code, div255_rn(r.v)) : r.v;
     }
 };
 

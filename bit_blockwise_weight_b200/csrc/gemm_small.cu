@@ -106,13 +106,16 @@ __device__ __forceinline__ uint32_t lut_off(uint32_t w, int j) {
     return sh & 0x7f80u;
 }
 
-// NT = 1 for M <= 8 (tokens 0..7), 2 for M <= 16
-template <typename D, int NT>
+// NT = 1 for M <= 8 (tokens 0..7), 2 for M <= 16.  GMODE: how absmax
+// arrives (0: 16-byte boxes by TMA; else the producer warp gathers it, see
+// below).
+template <typename D, int NT, int GMODE>
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_amx,
                   const __grid_constant__ CUtensorMap tmap_x, const AbsmaxSrc absmax,
                   const uint16_t *__restrict__ bias, uint16_t *__restrict__ Y, int M, int N, int K,
-                  int log2B, int amx_tma, int rbox, const __grid_constant__ CodeTable tab) {
+                  int log2B, int rbox, const __grid_constant__ CodeTable tab) {
+    constexpr bool amx_tma = GMODE == 0;
     extern __shared__ uint8_t smem_raw[];
     Smem &s = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~(uintptr_t)1023);
@@ -163,6 +166,37 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_const
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_w)) : "memory");
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_x)) : "memory");
         }
+        // Absmax rows not 16-byte pitched, or 8-bit statistics: the lanes
+        // gather each stage's scales themselves.  GMODE 1 (fp32) and 2 (8-bit
+        // codes of blocks of 64: one 32-bit word of four codes and one group
+        // scale per row) load a stage ahead into registers, and the values are
+        // finished when the stage is written, so the loads of stage q + 1 are
+        // in flight while the ring waits for a free slot.  GMODE 3 (other
+        // 8-bit layouts) gathers and finishes at the stage itself.
+        constexpr int GR = GMODE == 1 || GMODE == 2 ? kRowsMax / 32 : 1;
+        float gv[GR][GMODE == 1 ? RPS : 1];
+        uint32_t gw[GMODE == 2 ? GR : 1];
+        auto gather = [&](int q) {
+            const int b = b_lo + q * RPS;
+#pragma unroll
+            for (int pi = 0; pi < GR; ++pi) {
+                const int p = lane + 32 * pi;
+                if constexpr (GMODE == 1) {
+#pragma unroll
+                    for (int j = 0; j < RPS; ++j) {
+                        const int blk = ((b + j) * RUN) >> log2B;
+                        gv[pi][j] = (p < R && b + j < b_hi) ? __ldg(absmax.f32 + (int64_t)(r0 + p) * nblk + blk) : 0.0f;
+                    }
+                } else if constexpr (GMODE == 2) {
+                    // blocks b .. b + 3 of the row: four codes of one word, one group
+                    const int64_t f = (int64_t)(r0 + p) * nblk + b;
+                    const bool in = p < R && b < b_hi;
+                    gw[pi] = in ? __ldg(reinterpret_cast<const uint32_t *>(absmax.q + f)) : 0u;
+                    gv[pi][0] = in ? __ldg(absmax.scales + (f >> absmax.log2G)) : 0.0f;
+                }
+            }
+        };
+        if (GMODE != 0 && stages > 0) gather(0);
         int issued = 0;
         for (int q = 0; q < stages; ++q) {
             const int st = q % STAGES;
@@ -171,12 +205,34 @@ gemm_small_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_const
             if (!__all_sync(FULL, ok)) break;
             const int b = b_lo + q * RPS;                  // first run of the stage
             const int x0 = ((b * RUN) >> log2B) & ~3;      // first scale of the absmax box
-            if (!amx_tma)  // absmax rows not 16-byte pitched, or 8-bit statistics: gather the stage's scales
+            if constexpr (GMODE == 1) {
+#pragma unroll
+                for (int pi = 0; pi < GR; ++pi)
+#pragma unroll
+                    for (int j = 0; j < RPS; ++j) {
+                        const int p = lane + 32 * pi;
+                        const int blk = ((b + j) * RUN) >> log2B;
+                        if (p < R && b + j < b_hi) s.amx[st][p * 4 + (blk - x0)] = gv[pi][j];
+                    }
+            } else if constexpr (GMODE == 2) {
+#pragma unroll
+                for (int pi = 0; pi < GR; ++pi) {
+                    const int p = lane + 32 * pi;
+                    if (p < R) {
+                        const float step = div255_rn(gv[pi][0]);
+#pragma unroll
+                        for (int j = 0; j < RPS; ++j)
+                            if (b + j < b_hi) s.amx[st][p * 4 + j] = __fmul_rn((float)((gw[pi] >> (8 * j)) & 255u), step);
+                    }
+                }
+            } else if constexpr (GMODE == 3) {
                 for (int p = lane; p < R; p += 32)
                     for (int j = 0; j < RPS && b + j < b_hi; ++j) {
                         const int blk = ((b + j) * RUN) >> log2B;
                         s.amx[st][p * 4 + (blk - x0)] = absmax((int64_t)(r0 + p) * nblk + blk);
                     }
+            }
+            if (GMODE != 0 && q + 1 < stages) gather(q + 1);
             __syncwarp();  // the gathered scales are written before lane 0 arrives
             if (lane == 0) {
                 mbar_arrive_expect_tx(&s.full[st], tx);
@@ -311,7 +367,13 @@ template <typename D, int NT>
 cudaError_t set_smem_attr() {
     static std::atomic<bool> done[kMaxDevices];  // per device: attributes belong to a device's context
     return once_per_device(done, [] {
-        return cudaFuncSetAttribute(gemm_small_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+        const void *k[4] = {(const void *)gemm_small_kernel<D, NT, 0>, (const void *)gemm_small_kernel<D, NT, 1>,
+                            (const void *)gemm_small_kernel<D, NT, 2>, (const void *)gemm_small_kernel<D, NT, 3>};
+        for (const void *f : k) {
+            const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     });
 }
 
@@ -340,7 +402,7 @@ int cluster_capacity(int S) {
         cudaLaunchAttribute attr[1];
         cudaLaunchConfig_t cfg = make_cfg(dim3(1, 1, S), S, 0, attr);
         if (set_smem_attr<D, NT>() != cudaSuccess ||
-            cudaOccupancyMaxActiveClusters(&n, gemm_small_kernel<D, NT>, &cfg) != cudaSuccess || n <= 0) {
+            cudaOccupancyMaxActiveClusters(&n, gemm_small_kernel<D, NT, 0>, &cfg) != cudaSuccess || n <= 0) {
             (void)cudaGetLastError();
             n = device_sm_count() / S;
         }
@@ -405,9 +467,26 @@ cudaError_t launch_t(const void *X, const uint8_t *W, const AbsmaxSrc &absmax, c
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = make_cfg(dim3(plan.G, 1, plan.S), plan.S, stream, attr);
-    return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT>, map_w, map_amx, map_x, absmax,
-                              static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(Y), M, N, K,
-                              log2B, amx_tma, rbox, tab);
+    // absmax gathered by the producer: fp32 (1); 8-bit codes of blocks of 64
+    // with rows of whole 4-code words and groups of at least 4 (2); other
+    // 8-bit layouts (3)
+    const int gmode = amx_tma ? 0 : !absmax.q ? 1 : (log2B == 6 && nblk % 4 == 0 && absmax.log2G >= 2) ? 2 : 3;
+    const uint16_t *b16 = static_cast<const uint16_t *>(bias);
+    uint16_t *y16 = static_cast<uint16_t *>(Y);
+    switch (gmode) {
+    case 0:
+        return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT, 0>, map_w, map_amx, map_x, absmax, b16, y16, M, N,
+                                  K, log2B, rbox, tab);
+    case 1:
+        return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT, 1>, map_w, map_amx, map_x, absmax, b16, y16, M, N,
+                                  K, log2B, rbox, tab);
+    case 2:
+        return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT, 2>, map_w, map_amx, map_x, absmax, b16, y16, M, N,
+                                  K, log2B, rbox, tab);
+    default:
+        return cudaLaunchKernelEx(&cfg, gemm_small_kernel<D, NT, 3>, map_w, map_amx, map_x, absmax, b16, y16, M, N,
+                                  K, log2B, rbox, tab);
+    }
 }
 
 }  // namespace

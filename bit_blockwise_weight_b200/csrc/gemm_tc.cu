@@ -200,6 +200,36 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                 asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_amx))
                              : "memory");
         }
+        // Without absmax boxes (rows not 16-byte pitched, or 8-bit
+        // statistics) the lanes gather each stage's scales into the same
+        // [row][4] layout the tensor map would produce, one stage ahead: the
+        // loads of stage i + 1 are in flight while the ring waits for a slot.
+        // Element p (lane + 32 pi) of a stage: forward, row c0 + p of the
+        // stage's block; backward, row it BK + (p & 63), block column p >> 6.
+        AbsmaxRaw gv[8];
+        auto slot_of = [&](int it, int p, int &row, int &blk, int &at) {
+            if (BWD) {
+                row = it * BK + (p & 63);
+                blk = (c0 + 64 * (p >> 6)) >> log2B;
+                at = (p & 63) * 4 + (blk - bwd_x0);
+            } else {
+                row = c0 + p;
+                blk = (it * BK) >> log2B;
+                at = p * 4 + (blk & 3);
+            }
+        };
+        auto gather = [&](int i) {
+            const int it = i_lo + i;
+#pragma unroll
+            for (int pi = 0; pi < 8; ++pi) {
+                const int p = lane + 32 * pi;
+                int row, blk, at;
+                slot_of(it, p, row, blk, at);
+                const bool in = BWD ? (row < N && blk < nblk) : (p < BN && row < N);
+                gv[pi] = in ? absmax.raw((int64_t)row * nblk + blk) : AbsmaxRaw{0u, 0.0f};
+            }
+        };
+        if (!amx_tma && iters > 0) gather(0);
         int issued = 0;
         for (int i = 0; i < iters; ++i) {
             const int st = i % W_STAGES;
@@ -208,24 +238,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
             if (!__all_sync(FULL, ok)) break;
             const int it = i_lo + i;
             if (!amx_tma) {
-                // gather the stage's scales into the same [row][4] layout the
-                // tensor map would produce
                 float *dst = s.amx[st];
-                for (int p = lane; p < 256; p += 32) {
-                    int row, blk, idx;
-                    if (BWD) {
-                        row = it * BK + (p & 63);
-                        blk = (c0 + 64 * (p >> 6)) >> log2B;
-                        idx = blk - bwd_x0;
-                        if (p < 64 * 4) dst[(p & 63) * 4 + idx] =
-                            (row < N && blk < nblk) ? absmax((int64_t)row * nblk + blk) : 0.0f;
-                    } else {
-                        row = c0 + p;
-                        blk = (it * BK) >> log2B;
-                        idx = blk & 3;
-                        if (p < BN) dst[p * 4 + idx] = row < N ? absmax((int64_t)row * nblk + blk) : 0.0f;
-                    }
+#pragma unroll
+                for (int pi = 0; pi < 8; ++pi) {
+                    const int p = lane + 32 * pi;
+                    int row, blk, at;
+                    slot_of(it, p, row, blk, at);
+                    if (BWD || p < BN) dst[at] = absmax.finish(gv[pi]);
                 }
+                if (i + 1 < iters) gather(i + 1);
             }
             if (lane == 0) {
                 mbar_arrive_expect_tx(&s.full_w[st], tx);

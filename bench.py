@@ -37,6 +37,7 @@ sys.path.insert(0, ROOT)
 
 N_ELEMS = 1 << 28
 BLOCK = 64
+CLOCK_MHZ_NOMINAL = 1965   # B200 maximum SM clock (the fp32 FMA rate is computed at it)
 GEMV_SHAPES = [(4096, 4096), (4096, 1024), (4096, 14336), (14336, 4096)]
 SMALLM_SHAPES = [(8192, 28672), (28672, 8192)]
 SMALLM_M = 16
@@ -602,6 +603,45 @@ def time_next_rows(step, dev, hbm):
         out[name] = {"us": round(t32, 2)}
         dqn = name.replace("gemm_4bit", "gemm_4bit_dq", 1)
         out[dqn] = {"us": round(tdq, 2), "speedup_vs_fp32_absmax": round(t32 / tdq, 3)}
+    # fp32 compute dtype (x, bias and y in float32; CUDA-core FMAs on the exact
+    # fp32 dequantized weight): the decode shapes, M = 16 on the 70B shapes and
+    # prefill M = 512 forward / backward.  The prefill is compute-bound on the
+    # CUDA cores: its fraction is of the fp32 FMA rate from the unit counts
+    # (148 SMs x 128 lanes x 2 flops x the clock seen)
+    fp32_peak = 148 * 128 * 2 * CLOCK_MHZ_NOMINAL * 1e6 / 1e12
+    for K, N, p, a, xv, bias, y in step.gemv:
+        nb = N * K // BLOCK
+        C = copies_for(N * K // 2 + 4 * nb)
+        ps = [p] + [p.clone() for _ in range(C - 1)]
+        as_ = [a] + [a.clone() for _ in range(C - 1)]
+        x32, b32 = xv.float(), bias.float()
+        y32 = torch.empty(N, dtype=torch.float32, device=dev)
+        rec(f"gemv_4bit_f32_{K}x{N}", graph_per_launch(dev, [
+            lambda i=i: b.gemv_4bit(x32, ps[i], as_[i], N, K, b32, BLOCK, "nf4", out=y32) for i in range(C)]),
+            N * K // 2 + 4 * nb + 4 * K + 8 * N)
+        del ps, as_
+    for K, N, p, a, X, Y in step.smallm:
+        nb = N * K // BLOCK
+        ps = [p, p.clone()]
+        as_ = [a, a.clone()]
+        M = X.shape[0]
+        X32 = X.float()
+        Y32 = torch.empty(M, N, dtype=torch.float32, device=dev)
+        rec(f"gemm_4bit_f32_M{M}_{K}x{N}", graph_per_launch(dev, [
+            lambda i=i: b.gemm_4bit(X32, ps[i], as_[i], N, None, BLOCK, "nf4", out=Y32) for i in range(2)]),
+            N * K // 2 + 4 * nb + 4 * M * K + 4 * M * N)
+        del ps, as_
+    M, K, N, p, a, X, dY, Y, dX = step.prefill
+    X32, dY32 = X.float(), dY.float()
+    Y32 = torch.empty(M, N, dtype=torch.float32, device=dev)
+    dX32 = torch.empty(M, K, dtype=torch.float32, device=dev)
+    flops = 2.0 * M * N * K
+    for name, f in ((f"gemm_4bit_f32_M{M}_{K}x{N}", lambda: b.gemm_4bit(X32, p, a, N, None, BLOCK, "nf4", out=Y32)),
+                    (f"gemm_4bit_backward_f32_M{M}_{K}x{N}",
+                     lambda: b.gemm_4bit_backward(dY32, p, a, K, BLOCK, "nf4", out=dX32))):
+        us = graph_per_launch(dev, [f] * 2, reps=2)
+        tf = flops / (us / 1e6) / 1e12
+        out[name] = {"us": round(us, 2), "TFLOP/s": round(tf, 1), "fp32_fma_frac": round(tf / fp32_peak, 4)}
     out["note"] = ("each op alone, back to back in one CUDA graph over rotating copies of its inputs "
                    "(working set above 5x L2; the prefill ops reuse one 33 MB weight, compute-bound)")
     return out

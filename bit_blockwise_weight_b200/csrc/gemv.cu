@@ -87,6 +87,9 @@ namespace {
 constexpr int kWarps = BNB4_GEMV_WARPS;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSpan = BNB4_GEMV_SPAN;     // segments per group
+#ifndef BNB4_GEMV_PDL
+#define BNB4_GEMV_PDL 1                   // programmatic dependent launch (prologue overlaps the previous kernel)
+#endif
 #ifndef BNB4_GEMV_ILV
 #define BNB4_GEMV_ILV 2
 #endif
@@ -309,8 +312,10 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
     const int q_last = ng > 0 ? (g_hi - 1) / SS : -1;
 
     Unit ua[kSpan], ub[kSpan];
+#if !BNB4_GEMV_PDL
     // the first group's loads leave before the table and x are staged
     if (ng > 0) load(cq, css, ua);
+#endif
     {
         // table: entry v (codes of nibbles v >> 4, v & 15) copied to words 64 v + l, l < 32
         for (int idx = tid; idx < 2048; idx += kThreads) {   // 2048 16-byte pieces
@@ -319,6 +324,16 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
             sts128(lut_a + v * 256 + q * 16, make_uint4(e, e, e, e));
         }
         if (tid < kZero / 16) sts128(zero_a + 16 * tid, make_uint4(0, 0, 0, 0));
+#if BNB4_GEMV_PDL
+        // Launched as a programmatic dependent, this CTA may start while the
+        // previous kernel on the stream is still finishing: the work above
+        // reads only this kernel's parameters.  Every global access (inputs
+        // the previous kernel may write, y it may read) comes after the wait,
+        // which returns once that kernel has completed and its writes are
+        // visible.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (ng > 0) load(cq, css, ua);
+#endif
         // x: 16-byte piece q of item i at position (q + 2 (i & 1)) & 7 of the
         // item's 128 bytes; zeros past K.  All of a thread's loads leave before
         // any store, so staging costs one round trip.
@@ -449,6 +464,11 @@ gemv_kernel(const uint16_t *__restrict__ x, const uint8_t *__restrict__ W, const
             css = nss;
         }
     }
+#if BNB4_GEMV_PDL
+    // the next kernel on the stream may launch now (its CTAs take SMs as this
+    // grid's leave, and wait for its completion before touching memory)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
     __syncthreads();
 
     for (int r = tid; r < R; r += kThreads) {
@@ -513,10 +533,18 @@ cudaError_t launch_t(const void *x, const uint8_t *W, const void *absmax, const 
         return cudaFuncSetAttribute(gemv_kernel<D, DQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smax);
     });
     if (e != cudaSuccess) return e;
-    gemv_kernel<D, DQ><<<G, kThreads, smem_bytes(K, reserved), stream>>>(
-        static_cast<const uint16_t *>(x), W, absmax, scales, log2G, static_cast<const uint16_t *>(bias),
-        static_cast<uint16_t *>(y), N, K, log2B, tab);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem_bytes(K, reserved);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = BNB4_GEMV_PDL;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_kernel<D, DQ>, static_cast<const uint16_t *>(x), W, absmax, scales, log2G,
+                              static_cast<const uint16_t *>(bias), static_cast<uint16_t *>(y), N, K, log2B, tab);
 }
 
 }  // namespace

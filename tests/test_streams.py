@@ -122,3 +122,37 @@ def test_two_streams_on_disjoint_buffers_at_once():
         back = oracle.dequant_absmax(oq, osc, 256)
         ref = oracle.matmul(Xs, dt, op, back, None, M, N, K, B, "nf4")
         assert rel_l2(as_f64(to_host(Y), dt).reshape(M, N), ref) <= MATMUL_TOL
+
+
+def test_chained_gemvs_read_the_previous_output():
+    """Twenty gemv launches back to back, each reading the one before it as its
+    x (4096 -> 1024 -> 4096 ...), no host synchronisation.  The gemv may start
+    before the previous kernel ends (programmatic dependent launch); it must
+    still read that kernel's finished output.  Each step is compared with the
+    oracle applied to the previous step's GPU output."""
+    K1, N1 = 4096, 1024
+    B = 64
+    ws = []
+    for (N, K, seed) in ((N1, K1, 31), (K1, N1, 32)):
+        w = synthetic.weight(N, K, seed, sigma=1.0 / np.sqrt(K)).numpy().reshape(-1)
+        p, a = oracle.quantize(w, "f32", B, "nf4")
+        ws.append((N, K, p, a, torch.from_numpy(p).cuda(), torch.from_numpy(a).cuda()))
+    v0 = synthetic.activations(1, K1, seed=33).reshape(-1).cuda()
+    outs = []
+    x = v0
+    torch.cuda.synchronize()
+    torch.cuda._sleep(SPIN)                  # the chain queues up behind a long kernel
+    for i in range(20):
+        N, K, p, a, dp, da = ws[i % 2]
+        y = torch.empty(N, dtype=torch.bfloat16, device="cuda")
+        bnb4.gemv_4bit(x, dp, da, N, K, None, B, "nf4", out=y)
+        outs.append(y)
+        x = y
+    torch.cuda.synchronize()
+    prev = synthetic.storage_numpy(v0.cpu())
+    for i, y in enumerate(outs):
+        N, K, p, a, _, _ = ws[i % 2]
+        ref = oracle.matmul(prev, "bf16", p, a, None, 1, N, K, B, "nf4")[0]
+        got = to_host(y)
+        assert rel_l2(as_f64(got, "bf16"), ref) <= MATMUL_TOL, i
+        prev = got

@@ -10,8 +10,9 @@
 //   forward   D[M, N] = A[M, K] . W[N, K]^T   (A = X,  reduction over K)
 //   backward  D[M, K] = A[M, N] . W[N, K]     (A = dY, reduction over N)
 //
-// One CTA computes a 256 x BN output tile (BN = 256, or 224 when that fills
-// the SMs better) as two M=128 tcgen05.mma accumulators (2 x BN TMEM columns)
+// One CTA computes a 256 x BN output tile (BN = 256, or forward a narrower
+// multiple of 16 down to 160 when that fills the SMs better) as two M=128
+// tcgen05.mma accumulators (2 x BN TMEM columns)
 // that share one B operand:
 //   * warp 0, one thread: TMA loads of A (two 128 x 64 boxes per stage,
 //     128-byte swizzle) into a 3-slot ring;
@@ -53,7 +54,7 @@ namespace bnb4 {
 namespace {
 
 constexpr int BM = 256;           // two M=128 accumulators
-constexpr int BN_MAX = 256;       // output columns per tile (256, or 224 to fill the SMs)
+constexpr int BN_MAX = 256;       // output columns per tile (256, or narrower to fill the SMs)
 constexpr int BK = 64;            // reduction per stage (one 128-byte swizzle row)
 constexpr int A_STAGES = 3;
 constexpr int B_STAGES = 2;
@@ -425,7 +426,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant
                 const uint32_t tbase = tmem + mt * BN + ((uint32_t)(q * 32) << 16);
 #pragma unroll
                 for (int cc = 0; cc < RED_CW; cc += 16) {
-                    if (cb + cc >= BN) break;  // a 224-wide tile ends inside the last chunk
+                    if (cb + cc >= BN) break;  // a narrower tile ends inside the last chunk
                     uint32_t r[16];
                     tmem_ld16(tbase + cb + cc, r);
                     tmem_ld_wait();
@@ -534,9 +535,14 @@ cudaError_t launch_bn(const CUtensorMap &map_a, const CUtensorMap &map_w, const 
 }
 
 // Tile width and reduction split: the pair minimising
-//   waves x (stages per CTA + fixed cost) x width / 256,
+//   waves x (stages per CTA + fixed cost) x (kWidthFixed + width),
 // the fixed cost (prologue, epilogue; the cluster reduction when split) in
-// stage units.  A split keeps at least 8 stages per CTA.
+// stage units.  A stage's time grows with the width (the MMAs) on top of a
+// part that does not (the dequant warps convert all 256 rows of a stage
+// either way); measured on B200 at M = 2048, 160-wide tiles took 61 us per
+// wave and 256-wide 69 us, about 600 columns' worth of fixed time.  A split
+// keeps at least 8 stages per CTA.
+constexpr double kWidthFixed = 600.0;
 struct Plan {
     int bn, C;
 };
@@ -545,15 +551,15 @@ template <typename D, bool BWD>
 Plan make_plan(long mt, int n_out, int iters) {
     Plan best{256, 1};
     double best_t = 1e300;
-    for (int bn : {256, 224}) {
-        if (BWD && bn == 224) continue;  // the MN-major tile is built from 64-column atoms
+    for (int bn : {256, 224, 208, 192, 176, 160}) {
+        if (BWD && bn != 256) continue;  // the MN-major tile is built from 64-column atoms
         const long tiles = mt * ((n_out + bn - 1) / bn);
         for (int C = 1; C <= 8; C *= 2) {
             if (C > 1 && iters / C < 8) break;
-            const int cap = bn == 256 ? cluster_capacity<D, BWD, 256>(C)
-                                      : cluster_capacity<D, BWD, BWD ? 256 : 224>(C);
+            // residency does not depend on the width (shared memory is sized for 256)
+            const int cap = cluster_capacity<D, BWD, 256>(C);
             const long waves = (tiles * C + cap - 1) / cap;
-            const double t = (double)waves * ((iters + C - 1) / C + (C == 1 ? 4 : 8)) * bn / 256.0;
+            const double t = (double)waves * ((iters + C - 1) / C + (C == 1 ? 4 : 8)) * (kWidthFixed + bn);
             if (t < best_t - 1e-9) {
                 best_t = t;
                 best = Plan{bn, C};
@@ -604,9 +610,14 @@ cudaError_t launch_t(const void *A, const uint8_t *W, const AbsmaxSrc &absmax, c
         amx_tma = 0;
 
     if constexpr (!BWD) {
-        if (bn == 224)
-            return launch_bn<D, BWD, 224>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B,
-                                          amx_tma, tab, C, stream);
+        switch (bn) {
+        case 224: return launch_bn<D, BWD, 224>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma, tab, C, stream);
+        case 208: return launch_bn<D, BWD, 208>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma, tab, C, stream);
+        case 192: return launch_bn<D, BWD, 192>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma, tab, C, stream);
+        case 176: return launch_bn<D, BWD, 176>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma, tab, C, stream);
+        case 160: return launch_bn<D, BWD, 160>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma, tab, C, stream);
+        default: break;
+        }
     }
     return launch_bn<D, BWD, 256>(map_a, map_w, map_amx, absmax, bias, out, M, N, K, log2B, amx_tma,
                                   tab, C, stream);

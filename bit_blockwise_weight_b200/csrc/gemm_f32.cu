@@ -24,8 +24,8 @@
 //                     the step's weight tile is dequantized into shared memory
 //                     as fp32 (transposed for the forward, as stored for the
 //                     backward), the activations tile is staged beside it,
-//                     and each thread accumulates a 4 x 4 (BM = 64) or 1 x 4
-//                     (BM = 16) block of outputs.
+//                     and each thread accumulates a 4 x 4 block of outputs
+//                     (256 threads per 64-row tile, 64 per 16-row tile).
 //
 // No global scratch.
 #include <atomic>
@@ -178,16 +178,34 @@ gemv_f32_kernel(const float *__restrict__ x, const uint8_t *__restrict__ W, cons
 
 constexpr int kBN = 64;   // output columns per tile (weight rows forward, K columns backward)
 constexpr int kBK = 64;   // reduction step
-constexpr int kGThreads = 256;
+
+// cluster barrier and a load from another CTA's shared memory (split reduction)
+__device__ __forceinline__ void cluster_barrier() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t local_addr, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+    return v;
+}
 
 // BWD == false: Y[m, n] = sum_k A[m, k] W[n, k] (+ bias[n]), A = X [M, K], tile over (m, n), step over k.
 // BWD == true:  Y[m, k] = sum_n A[m, n] W[n, k], A = dY [M, N], tile over (m, k), step over n.
+// Every thread accumulates a 4 x 4 block (4 m x 4 output columns): per
+// reduction index two 16-byte shared loads feed 16 FMAs.  BM = 64 uses 256
+// threads per tile, BM = 16 (M <= 16) 64, several tiles per SM.  With
+// gridDim.z = S > 1 the S CTAs of a cluster split the reduction steps; their
+// partial tiles meet in shared memory and are added in rank order (the same
+// bits on every run), each rank storing a share of the tile's rows.
 template <int BM, bool BWD>
-__global__ void __launch_bounds__(kGThreads)
+__global__ void __launch_bounds__(BM * 4)
 gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, const float *__restrict__ absmax,
                 const float *__restrict__ bias, float *__restrict__ Y, int M, int N, int K, int log2B,
                 const __grid_constant__ CodeTable tab) {
-    constexpr int TM = BM / 16;                    // outputs per thread along m (4 or 1)
+    constexpr int TM = 4;                          // outputs per thread along m
+    constexpr int kGThreads = BM * 4;              // 16 column groups x BM / 4 row groups
     __shared__ __align__(16) float As[kBK][BM + 4];     // [reduction][m]
     __shared__ __align__(16) float Bs[kBK][kBN + 4];    // [reduction][output column]
     __shared__ float code[16];
@@ -197,7 +215,7 @@ gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, cons
     const int c0 = blockIdx.x * kBN;               // first output column of the tile
     const int ncols = BWD ? K : N;                 // output columns
     const int red = BWD ? N : K;                   // reduction length
-    const int tx = tid & 15, ty = tid >> 4;        // 16 x 16 threads: columns 4 tx.., rows TM ty..
+    const int tx = tid & 15, ty = tid >> 4;        // columns 4 tx .. 4 tx + 3, rows TM ty .. TM ty + 3
     const int64_t row_bytes = K >> 1;
     const int nblk = K >> log2B;
     float acc[TM][4];
@@ -205,16 +223,19 @@ gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, cons
     for (int i = 0; i < TM; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
     __syncthreads();
 
-    for (int r0 = 0; r0 < red; r0 += kBK) {
+    const int S = gridDim.z, z = blockIdx.z;
+    const int nsteps = (red + kBK - 1) / kBK;
+    const int st_lo = (int)(((int64_t)nsteps * z) / S), st_hi = (int)(((int64_t)nsteps * (z + 1)) / S);
+    for (int r0 = st_lo * kBK; r0 < st_hi * kBK; r0 += kBK) {
         // activations: A[m0 + i][r0 + j] -> As[j][i], zeros outside
         for (int e = tid; e < BM * kBK; e += kGThreads) {
             const int i = e / kBK, j = e % kBK;
             const int m = m0 + i, r = r0 + j;
             As[j][i] = (m < M && r < red) ? A[(int64_t)m * red + r] : 0.f;
         }
-        // weight tile: 64 weight rows x 64 weights, one thread per (row, 16 weights)
-        {
-            const int lr = tid >> 2, part = tid & 3;   // tile row, quarter of the 64 weights
+        // weight tile: 64 weight rows x 64 weights, in pieces of (row, 16 weights)
+        for (int pc = tid; pc < 256; pc += kGThreads) {
+            const int lr = pc >> 2, part = pc & 3;     // tile row, quarter of the 64 weights
             int wrow, wk;                               // weight row and first k of this thread's 16
             if (!BWD) { wrow = c0 + lr; wk = r0 + 16 * part; }
             else { wrow = r0 + lr; wk = c0 + 16 * part; }
@@ -241,9 +262,8 @@ gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, cons
         __syncthreads();
 #pragma unroll 8
         for (int j = 0; j < kBK; ++j) {
-            float a[TM];
-#pragma unroll
-            for (int i = 0; i < TM; ++i) a[i] = As[j][TM * ty + i];
+            const float4 aq = *reinterpret_cast<const float4 *>(&As[j][TM * ty]);
+            const float a[TM] = {aq.x, aq.y, aq.z, aq.w};
             const float4 bq = *reinterpret_cast<const float4 *>(&Bs[j][4 * tx]);
             const float b[4] = {bq.x, bq.y, bq.z, bq.w};
 #pragma unroll
@@ -253,19 +273,45 @@ gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, cons
         }
         __syncthreads();
     }
+    if (S == 1) {
 #pragma unroll
-    for (int i = 0; i < TM; ++i) {
-        const int m = m0 + TM * ty + i;
-        if (m >= M) continue;
+        for (int i = 0; i < TM; ++i) {
+            const int m = m0 + TM * ty + i;
+            if (m >= M) continue;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int col = c0 + 4 * tx + c;
-            if (col >= ncols) continue;
-            float v = acc[i][c];
+            for (int c = 0; c < 4; ++c) {
+                const int col = c0 + 4 * tx + c;
+                if (col >= ncols) continue;
+                float v = acc[i][c];
+                if (!BWD && bias) v += bias[col];
+                Y[(int64_t)m * ncols + col] = v;
+            }
+        }
+        return;
+    }
+    // split: this CTA's partial tile [BM][kBN] in the (now idle) A tile, then
+    // rank z adds rows [BM z / S, BM (z+1) / S) over the ranks in order
+    static_assert(BM * kBN <= kBK * (BM + 4), "partial tile fits in the A tile");
+    float *Ps = &As[0][0];
+#pragma unroll
+    for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) Ps[(TM * ty + i) * kBN + 4 * tx + c] = acc[i][c];
+    cluster_barrier();
+    const int rlo = (BM * z) / S, rhi = (BM * (z + 1)) / S;
+    const uint32_t ps_addr = (uint32_t)__cvta_generic_to_shared(Ps);
+    for (int e = tid; e < (rhi - rlo) * kBN; e += kGThreads) {
+        const int lr = rlo + e / kBN, lc = e % kBN;
+        const uint32_t la = ps_addr + (uint32_t)(lr * kBN + lc) * 4u;
+        float v = 0.f;
+        for (int q = 0; q < S; ++q) v += ld_cluster_f32(la, (uint32_t)q);
+        const int m = m0 + lr, col = c0 + lc;
+        if (m < M && col < ncols) {
             if (!BWD && bias) v += bias[col];
             Y[(int64_t)m * ncols + col] = v;
         }
     }
+    cluster_barrier();  // no CTA leaves while its partial tile may still be read
 }
 
 size_t gemv_f32_smem(int K) {
@@ -302,24 +348,31 @@ cudaError_t launch_gemm_f32(const float *A, const uint8_t *W, const float *absma
     const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
     const int ncols = (int)(backward ? K : N);
     const int log2B = ilog2(blocksize);
-    if (M <= 16) {
-        const dim3 grid((ncols + kBN - 1) / kBN, (unsigned)((M + 15) / 16));
-        if (backward)
-            gemm_f32_kernel<16, true><<<grid, kGThreads, 0, stream>>>(A, W, absmax, nullptr, Y, (int)M, (int)N,
-                                                                     (int)K, log2B, tab);
-        else
-            gemm_f32_kernel<16, false><<<grid, kGThreads, 0, stream>>>(A, W, absmax, bias, Y, (int)M, (int)N,
-                                                                      (int)K, log2B, tab);
-    } else {
-        const dim3 grid((ncols + kBN - 1) / kBN, (unsigned)((M + 63) / 64));
-        if (backward)
-            gemm_f32_kernel<64, true><<<grid, kGThreads, 0, stream>>>(A, W, absmax, nullptr, Y, (int)M, (int)N,
-                                                                     (int)K, log2B, tab);
-        else
-            gemm_f32_kernel<64, false><<<grid, kGThreads, 0, stream>>>(A, W, absmax, bias, Y, (int)M, (int)N,
-                                                                      (int)K, log2B, tab);
+    // reduction split S (a cluster of S CTAs along z): enough CTAs for about
+    // 4 per SM, at least 8 reduction steps each, S a power of two up to 8
+    const int BM = M <= 16 ? 16 : 64;
+    const int64_t tiles = (int64_t)((ncols + kBN - 1) / kBN) * ((M + BM - 1) / BM);
+    const int nsteps = (int)((backward ? N : K) + kBK - 1) / kBK;
+    int S = 1;
+    while (S < 8 && tiles * S < 4LL * device_sm_count() && nsteps / (2 * S) >= 8) S *= 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((ncols + kBN - 1) / kBN, (unsigned)((M + BM - 1) / BM), S);
+    cfg.blockDim = dim3(BM * 4, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = S;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int m = (int)M, n = (int)N, k = (int)K;
+    if (BM == 16) {
+        if (backward) return cudaLaunchKernelEx(&cfg, gemm_f32_kernel<16, true>, A, W, absmax, (const float *)nullptr, Y, m, n, k, log2B, tab);
+        return cudaLaunchKernelEx(&cfg, gemm_f32_kernel<16, false>, A, W, absmax, bias, Y, m, n, k, log2B, tab);
     }
-    return cudaGetLastError();
+    if (backward) return cudaLaunchKernelEx(&cfg, gemm_f32_kernel<64, true>, A, W, absmax, (const float *)nullptr, Y, m, n, k, log2B, tab);
+    return cudaLaunchKernelEx(&cfg, gemm_f32_kernel<64, false>, A, W, absmax, bias, Y, m, n, k, log2B, tab);
 }
 
 }  // namespace bnb4

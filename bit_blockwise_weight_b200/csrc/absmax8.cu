@@ -38,6 +38,9 @@ double_quant_kernel(const float *__restrict__ absmax, int64_t n, int log2G, uint
     for (int64_t g = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5); g < ngroups; g += warps) {
         const int64_t g0 = g << log2G;
         float m = 0.0f;
+        // unrolled, so a lane's loads of the group leave together instead of
+        // each waiting for the comparison before it
+#pragma unroll 8
         for (int j = lane; j < G; j += 32) {
             const int64_t i = g0 + j;
             if (i < n) {
@@ -51,6 +54,7 @@ double_quant_kernel(const float *__restrict__ absmax, int64_t n, int log2G, uint
             if (v > m) m = v;
         }
         if (lane == 0) scales[g] = m;
+#pragma unroll 8
         for (int j = lane; j < G; j += 32) {
             const int64_t i = g0 + j;
             if (i >= n) break;

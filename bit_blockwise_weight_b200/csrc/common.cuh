@@ -145,17 +145,25 @@ constexpr float kNear = 0x1p-19f;
 
 QuantTables host_quant_tables(bnb4_quant_type qt);
 
+// FP4 screen tables for inputs whose significands have p bits (bf16: 8,
+// fp16: 11), with which the one-shuffle screen decides every element exactly
+// (no element is near a threshold; see tables.cu).  Returns false, leaving
+// q unusable, if a key cannot be placed.
+bool host_fp4_exact_tables(int p, QuantTables &q);
+
 // 12582925 = 1.5 * 2^23 + 13: the fma lands in [2^23, 2^24) where the fp32
 // spacing is 1, so the low mantissa bits hold rn(13 v + 13).
 __device__ __forceinline__ uint32_t cell_of(float v) {
     return __float_as_uint(__fmaf_rn(v, 13.0f, 12582925.0f));
 }
 
+// NaN gives index 0, as a search for the smallest distance that never
+// improves on entry 0
 __device__ __forceinline__ uint32_t nearest_code(float v, float my_thr, uint32_t my_lohi) {
     uint32_t k = cell_of(v);
     float t = __shfl_sync(FULL, my_thr, k);   // shfl reads lane k & 31
     uint32_t lh = __shfl_sync(FULL, my_lohi, k);
-    return (v > t) ? (lh >> 4) : (lh & 15u);
+    return v != v ? 0u : (v > t) ? (lh >> 4) : (lh & 15u);
 }
 
 // ------------------------------------------------------------- helpers

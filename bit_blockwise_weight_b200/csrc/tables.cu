@@ -1,6 +1,7 @@
 // tables.cu -- host construction of the code tables and of the decision
 // tables that the quantize kernel searches (see common.cuh).
 #include <cmath>
+#include <cstdint>
 #include <cstdlib>
 #include <cstring>
 
@@ -108,6 +109,66 @@ QuantTables host_quant_tables(bnb4_quant_type qt) {
     }
     q.fast = !ok ? 0 : ident ? 1 : fold ? 2 : 0;
     return q;
+}
+
+// FP4 with 16-bit inputs.  The codes are E2M1 / 6, so the nominal decision
+// points are T = k / 24 (k in {1, 3, 5, 7, 10, 14, 20}, either sign); the
+// fp32 codes move each midpoint from T by about 1e-9.  For x and a with p-bit
+// significands (x = X 2^ex, a = A 2^ea, X, A < 2^p, a >= 2^(ea+p-1) when
+// normal), 24 x - k a is a multiple of 2^min(ex, ea), so a ratio x / a that
+// is not exactly T lies at least 2^(min(ex, ea) - ea - p) / 24 from it; near
+// T, x / a < 2^(ex - ea + 1) forces ex - ea >= e_T, the smallest integer
+// above log2 |T| - 1, which gives the gap g_T = 2^(e_T - p) / 24 (a
+// subnormal a only widens it).  So every element is either exactly on T or
+// at least g_T away, and a key placed about g_T / 2 from T, on the side that
+// sends an exact tie where the IEEE quotient RN(T) sends it, decides every
+// element of a block with absmax in the screen's range: the screen's own
+// error, with r = RN(1/a) from the exact reciprocal, is below |x / a| 2^-24.
+// The key keeps the rank above in its low mantissa nibble (a shift of at
+// most 8 ulps, inside the margins checked below).
+bool host_fp4_exact_tables(int p, QuantTables &q) {
+    q = host_quant_tables(BNB4_FP4);
+    if (!q.valid || q.fast != 2) return false;
+    // the distinct values in rank order, as numerators over 12
+    static const int n12[15] = {-12, -8, -6, -4, -3, -2, -1, 0, 1, 2, 3, 4, 6, 8, 12};
+    const CodeTable c = host_code_table(BNB4_FP4);
+    float val[15];
+    for (int r = 0; r < 15; ++r) {
+        val[r] = (float)(n12[r] / 12.0);
+        bool found = false;
+        for (int i = 0; i < 16; ++i) found |= c.v[i] == val[r];
+        if (!found) return false;  // the codes are these values rounded once
+    }
+    for (int k = 0; k < 32; ++k) {
+        if (q.thr[k] == 2.0f) continue;  // no threshold in the cell: the key stays below every value
+        const int R = (int)((q.rank_lohi[k] >> 4) & 15u);  // rank just above the threshold
+        if (R < 1 || R > 14) return false;
+        const double T = (n12[R - 1] + n12[R]) / 24.0;
+        const double mid = 0.5 * ((double)val[R - 1] + (double)val[R]);
+        // an exact tie x / a == T has the IEEE quotient RN(T) (T is not a
+        // float midpoint), which goes above the threshold iff RN(T) > thr
+        const bool up = (float)T > q.thr[k];
+        const int e = (int)std::floor(std::log2(std::fabs(T)) - 1.0 - 1e-9) + 1;
+        const double gap = std::ldexp(1.0, e - p) / 24.0;
+        const double err = std::fabs(T) * 0x1p-24 * (1.0 + 0x1p-20) + 0x1p-60;
+        if (std::fabs(mid - T) > gap / 64) return false;
+        float K = (float)(up ? T - gap / 2 : T + gap / 2);
+        uint32_t kb;
+        std::memcpy(&kb, &K, 4);
+        int64_t cand = (int64_t)((kb & ~15u) | (uint32_t)R);
+        if (cand - (int64_t)kb > 8) cand -= 16;
+        if ((int64_t)kb - cand > 8) cand += 16;
+        kb = (uint32_t)cand;
+        std::memcpy(&K, &kb, 4);
+        const double Kd = K;
+        // ties and every other ratio stay on their sides of the key, with
+        // room for the screen's error
+        if (up ? !(Kd > T - gap + err && Kd < T - err) : !(Kd > T + err && Kd < T + gap - err)) return false;
+        for (int j = 0; j <= 26; ++j)  // and the cell is still exact
+            if (std::fabs(Kd - (j - 12.5) / 13.0) <= 0x1p-16) return false;
+        q.key[k] = kb;
+    }
+    return true;
 }
 
 }  // namespace bnb4

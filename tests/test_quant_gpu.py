@@ -99,6 +99,69 @@ def test_special_values():
         assert gp[-1] & 15 == 0, "odd tail keeps the low nibble 0"
 
 
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("q", ["nf4", "fp4"])
+def test_nan_and_inf_elements(q, dtype):
+    """NaN is skipped by the maximum and gets index 0; an infinite element makes
+    absmax infinite, so the block's finite elements normalise to 0 and the
+    infinite ones to NaN (index 0)."""
+    tdt = synthetic.TORCH_DTYPES[dtype]
+    x = synthetic.roundtrip_tensor(64 * 40 + 9, seed=17, dtype=dtype).float()
+    x[5] = float("nan")                     # a NaN among ordinary values
+    x[64 * 3: 64 * 4: 7] = float("nan")     # several in one block
+    x[64 * 6: 64 * 7] = float("nan")        # a block of NaN only: absmax 0
+    x[64 * 9 + 3] = float("inf")
+    x[64 * 12 + 60] = -float("inf")
+    x[64 * 15 + 1] = float("nan")
+    x[64 * 15 + 2] = float("inf")
+    x[-4] = float("nan")                    # in the ragged tail
+    xs = synthetic.storage_numpy(x.to(tdt))
+    for B in (64, 256):
+        gp, ga = _gpu_quant(xs, dtype, B, q)
+        op, oa = oracle.quantize(xs, dtype, B, q)
+        assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32)), ("absmax", B)
+        bad = np.nonzero(gp != op)[0]
+        assert bad.size == 0, (B, bad.size, bad[:4])
+
+
+def _fp4_ratio_ties(n, B, dtype, seed):
+    """Blocks whose elements are the block's absmax times each FP4 decision point
+    k / 24, rounded to the input dtype (often exact: x / a lands on the point),
+    with a third of them moved one step of the dtype either way, random signs,
+    absmax over a wide exponent range, zeros and a NaN in some blocks."""
+    tdt = synthetic.TORCH_DTYPES[dtype]
+    g = torch.Generator().manual_seed(seed)
+    nb = -(-n // B)
+    lo, hi = (-40, 40) if dtype == "bf16" else (-12, 12)
+    a = ((torch.rand(nb, generator=g) * 4 + 0.25) * 2.0 ** torch.randint(lo, hi, (nb,), generator=g).float())
+    a = a.to(tdt).float()
+    k = torch.tensor([0, 1, 3, 5, 7, 10, 14, 20, 24], dtype=torch.float32)
+    x = (a[:, None] * k[torch.randint(0, len(k), (nb, B), generator=g)] / 24).to(tdt)
+    step = torch.randint(-1, 2, (nb, B), generator=g).to(torch.int16)
+    moved = (x.view(torch.int16) + step).view(tdt)
+    x = torch.where((torch.rand(nb, B, generator=g) < 0.3) & (x != 0), moved, x)
+    x = x * torch.where(torch.rand(nb, B, generator=g) < 0.5, -1.0, 1.0).to(tdt)
+    x[:, 0] = a.to(tdt)
+    nan_blocks = torch.rand(nb, generator=g) < 0.05
+    x[nan_blocks, B // 2] = float("nan")
+    return synthetic.storage_numpy(x.reshape(-1)[:n].contiguous())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("B", [64, 256, 4096])
+@pytest.mark.parametrize("n", [64, 4096 * 3 + 17, 1 << 20])
+def test_fp4_exact_ratio_ties(dtype, B, n):
+    """FP4 decision points are short fractions k / 24 that ratios of 16-bit
+    inputs hit exactly (and otherwise stay clear of by a fixed gap); each tie
+    must go where the IEEE quotient sends it."""
+    xs = _fp4_ratio_ties(n, B, dtype, seed=n % 101 + B)
+    gp, ga = _gpu_quant(xs, dtype, B, "fp4")
+    op, oa = oracle.quantize(xs, dtype, B, "fp4")
+    assert np.array_equal(ga.view(np.uint32), oa.view(np.uint32)), "absmax"
+    bad = np.nonzero(gp != op)[0]
+    assert bad.size == 0, (bad.size, bad[:4])
+
+
 def test_n_zero_is_a_noop():
     packed, absmax = bnb4.quantize_4bit(torch.empty(0, device="cuda"), 64, "nf4")
     assert packed.numel() == 0 and absmax.numel() == 0

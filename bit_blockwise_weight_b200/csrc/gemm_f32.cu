@@ -19,7 +19,8 @@
 //                     reduced across lanes when a warp leaves a quad; quads
 //                     that two warps share are added in warp order, so the
 //                     result is the same bits on every run.
-//   gemm_f32_kernel   M >= 2 and the backward.  A classic shared-memory tiled
+//   gemm_f32_smallm_kernel  2 <= M <= 16, forward (below).
+//   gemm_f32_kernel   M > 16 and the backward.  A classic shared-memory tiled
 //                     product: BM x 64 output tiles, 64-wide reduction steps;
 //                     the step's weight tile is dequantized into shared memory
 //                     as fp32 (transposed for the forward, as stored for the
@@ -51,6 +52,13 @@ __device__ __forceinline__ uint4 ldg_nc16(const void *p) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
+}
+
+// the value of `v` held by lane (lane_bits & 31)
+__device__ __forceinline__ uint32_t shfl_idx(uint32_t v, uint32_t lane_bits) {
+    uint32_t r;
+    asm volatile("shfl.sync.idx.b32 %0, %1, %2, 0x1f, 0xffffffff;" : "=r"(r) : "r"(v), "r"(lane_bits));
+    return r;
 }
 
 __global__ void __launch_bounds__(kVThreads, 1)
@@ -314,6 +322,234 @@ gemm_f32_kernel(const float *__restrict__ A, const uint8_t *__restrict__ W, cons
     cluster_barrier();  // no CTA leaves while its partial tile may still be read
 }
 
+// ------------------------------------------------- small M, forward
+//
+// M <= 16 (rows padded to MT): every weight is decoded once and meets all MT
+// rows of x in registers, and all lanes of a warp step through K together, so
+// each x value is one broadcast shared-memory read.  A CTA owns 128 TN weight
+// rows (thread i rows t * 128 + i, t < TN).  Per step of 128 weights the CTA
+// copies 64 contiguous bytes of each of its rows into shared memory
+// (asynchronous 16-byte copies, four threads per row) together with the
+// step's x, one step ahead of the arithmetic; a thread then reads its rows 16
+// bytes (32 weights) at a time (rows padded to 80 bytes: the reads of 8 lanes
+// fall in distinct banks), takes each code by a shuffle from a lane-held table
+// and multiplies it by the block's absmax (the exact fp32 weight).  56 KB of
+// shared memory leaves room for 4 CTAs per SM (measured on B200: 128-weight
+// steps beat 256-weight ones, which hold only 2).  With gridDim.z = S > 1 the
+// S CTAs of a cluster split K and add their partial tiles in rank order; S is
+// chosen for the fewest waves per unit of work.
+constexpr int kSMThreads = 128;
+constexpr int kSMStep = 128;                  // weights of a row per step
+constexpr int kSMRowPitch = kSMStep / 2 + 16; // bytes per staged row (padded by 16)
+constexpr int kSMPieces = kSMStep / 32;       // 16-byte pieces per row per step
+
+__host__ __device__ constexpr size_t sm_w_bytes(int TN) { return (size_t)kSMThreads * TN * kSMRowPitch; }
+__host__ __device__ constexpr size_t sm_x_bytes(int MT) { return (size_t)kSMStep * MT * sizeof(float); }
+__host__ __device__ constexpr size_t sm_smem(int MT, int TN) { return 2 * (sm_w_bytes(TN) + sm_x_bytes(MT)); }
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float *src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
+template <int MT, int TN>
+__global__ void __launch_bounds__(kSMThreads)
+gemm_f32_smallm_kernel(const float *__restrict__ X, const uint8_t *__restrict__ W, const float *__restrict__ absmax,
+                       const float *__restrict__ bias, float *__restrict__ Y, int M, int N, int K, int log2B,
+                       const __grid_constant__ CodeTable tab) {
+    static_assert(MT % 4 == 0 && MT <= 16, "rows in float4 groups");
+    constexpr int kRows = kSMThreads * TN;        // weight rows (output columns) per CTA
+    static_assert(MT * kRows * sizeof(float) <= sm_smem(MT, TN), "partial tile fits in the buffers");
+    // [2] weight stages [kRows][kSMRowPitch], then [2] x stages [kSMStep][MT];
+    // the partial tile at the end
+    extern __shared__ __align__(16) uint8_t smb[];
+    const uint32_t sm_a = (uint32_t)__cvta_generic_to_shared(smb);
+    const uint32_t w_a = sm_a, x_a = sm_a + 2 * (uint32_t)sm_w_bytes(TN);
+    const float *xsm = reinterpret_cast<const float *>(smb + 2 * sm_w_bytes(TN));
+    const int tid = threadIdx.x, lane = tid & 31;
+    const uint32_t my_code = __float_as_uint(tab.v[lane & 15]);
+    const int c0 = blockIdx.x * kRows;
+    const int S = gridDim.z, z = blockIdx.z;
+    const int n64 = K / 64;                       // K is a multiple of the blocksize (>= 64)
+    const int k_lo = (int)(((int64_t)n64 * z) / S) * 64;
+    const int k_hi = (int)(((int64_t)n64 * (z + 1)) / S) * 64;
+    const int64_t row_bytes = K >> 1;
+    const int nblk = K >> log2B;
+    const float *arow[TN];
+#pragma unroll
+    for (int t = 0; t < TN; ++t) arow[t] = absmax + (int64_t)min(c0 + t * kSMThreads + tid, N - 1) * nblk;
+    float acc[MT][TN];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int t = 0; t < TN; ++t) acc[m][t] = 0.f;
+
+    // one step's weights (the CTA's rows, 16-byte pieces of [kb, kb + kn)) and
+    // x (x[m][kb + kk] -> [kk][m], zeros past M and past kn); rows past N are
+    // clamped to the last one (their sums are never stored)
+    auto stage = [&](int kb, int buf) {
+        const int kn = min(kSMStep, k_hi - kb);
+        const int pieces = kn / 32;               // 16-byte pieces per row
+        for (int c = tid; c < kRows * kSMPieces; c += kSMThreads) {
+            const int r = c / kSMPieces, pc = c % kSMPieces;
+            if (pc < pieces) {
+                const int n = min(c0 + r, N - 1);
+                cp_async16(w_a + (uint32_t)(buf * sm_w_bytes(TN) + r * kSMRowPitch + 16 * pc),
+                           W + (int64_t)n * row_bytes + (kb >> 1) + 16 * pc);
+            }
+        }
+        for (int e = tid; e < MT * kSMStep; e += kSMThreads) {
+            const int m = e / kSMStep, kk = e % kSMStep;
+            const bool valid = m < M && kk < kn;
+            cp_async4(x_a + (uint32_t)(buf * sm_x_bytes(MT) + (kk * MT + m) * sizeof(float)),
+                      valid ? X + (int64_t)m * K + kb + kk : X, valid);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    if (k_lo < k_hi) stage(k_lo, 0);
+    int buf = 0;
+    for (int kb = k_lo; kb < k_hi; kb += kSMStep) {
+        if (kb + kSMStep < k_hi) {
+            stage(kb + kSMStep, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();  // every thread's copies of this step have landed
+        const int pieces = min(kSMStep, k_hi - kb) / 32;
+        const uint32_t wrow0 = w_a + (uint32_t)(buf * sm_w_bytes(TN) + tid * kSMRowPitch);
+        const float *xs = xsm + buf * (sm_x_bytes(MT) / sizeof(float));
+        for (int pc = 0; pc < pieces; ++pc) {
+            uint4 w[TN];
+            float a[TN];
+#pragma unroll
+            for (int t = 0; t < TN; ++t) {
+                w[t] = lds128(wrow0 + (uint32_t)(t * kSMThreads * kSMRowPitch + 16 * pc));
+                a[t] = __ldg(arow[t] + ((kb + 32 * pc) >> log2B));
+            }
+            // byte j holds reduction indices 2j (high nibble) and 2j + 1
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float wv[2][TN];
+#pragma unroll
+                for (int t = 0; t < TN; ++t) {
+                    const uint32_t wd = (j >> 2) == 0 ? w[t].x : (j >> 2) == 1 ? w[t].y : (j >> 2) == 2 ? w[t].z : w[t].w;
+                    const int sh = 8 * (j & 3);
+                    // the shuffle reads lane (index & 31); lanes 16..31 repeat the table
+                    wv[0][t] = __fmul_rn(__uint_as_float(shfl_idx(my_code, wd >> (sh + 4))), a[t]);
+                    wv[1][t] = __fmul_rn(__uint_as_float(shfl_idx(my_code, wd >> sh)), a[t]);
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float *xr = xs + (32 * pc + 2 * j + h) * MT;
+#pragma unroll
+                    for (int q = 0; q < MT / 4; ++q) {
+                        const float4 xv = *reinterpret_cast<const float4 *>(xr + 4 * q);
+#pragma unroll
+                        for (int t = 0; t < TN; ++t) {
+                            acc[4 * q][t] = __fmaf_rn(xv.x, wv[h][t], acc[4 * q][t]);
+                            acc[4 * q + 1][t] = __fmaf_rn(xv.y, wv[h][t], acc[4 * q + 1][t]);
+                            acc[4 * q + 2][t] = __fmaf_rn(xv.z, wv[h][t], acc[4 * q + 2][t]);
+                            acc[4 * q + 3][t] = __fmaf_rn(xv.w, wv[h][t], acc[4 * q + 3][t]);
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();  // this buffer is free for the step after next
+        buf ^= 1;
+    }
+    if (S == 1) {
+#pragma unroll
+        for (int t = 0; t < TN; ++t) {
+            const int n = c0 + t * kSMThreads + tid;
+            if (n >= N) continue;
+            const float bv = bias ? bias[n] : 0.f;
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M) Y[(int64_t)m * N + n] = bias ? acc[m][t] + bv : acc[m][t];
+        }
+        return;
+    }
+    // split: the partial tile [MT][kRows] in the buffers (idle since the last
+    // barrier), then rank z adds rows [MT z / S, MT (z+1) / S) over the ranks
+    // in order
+    float *ps = reinterpret_cast<float *>(smb);
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int t = 0; t < TN; ++t) ps[m * kRows + t * kSMThreads + tid] = acc[m][t];
+    cluster_barrier();
+    const int rlo = (MT * z) / S, rhi = (MT * (z + 1)) / S;
+    for (int e = tid; e < (rhi - rlo) * kRows; e += kSMThreads) {
+        const int m = rlo + e / kRows, col = e % kRows, n = c0 + col;
+        const uint32_t la = sm_a + (uint32_t)(m * kRows + col) * 4u;
+        float v = 0.f;
+        for (int q = 0; q < S; ++q) v += ld_cluster_f32(la, (uint32_t)q);
+        if (m < M && n < N) Y[(int64_t)m * N + n] = bias ? v + bias[n] : v;
+    }
+    cluster_barrier();  // no CTA leaves while its partial tile may still be read
+}
+
+template <int MT, int TN>
+cudaError_t launch_smallm(const float *A, const uint8_t *W, const float *absmax, const float *bias, float *Y, int M,
+                          int N, int K, int log2B, const CodeTable &tab, cudaStream_t stream) {
+    const int SMs = device_sm_count();
+    constexpr int kRows = kSMThreads * TN;
+    constexpr size_t smem = sm_smem(MT, TN);
+    static std::atomic<bool> set[kMaxDevices];
+    cudaError_t e = once_per_device(set, [] {
+        return cudaFuncSetAttribute(gemm_f32_smallm_kernel<MT, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)smem);
+    });
+    if (e != cudaSuccess) return e;
+    const int tiles = (N + kRows - 1) / kRows;
+    static std::atomic<int> occ_cache[kMaxDevices];
+    const int per_sm = cached_per_device(occ_cache, [] {
+        int v = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, gemm_f32_smallm_kernel<MT, TN>, kSMThreads, smem) !=
+                cudaSuccess || v < 1) {
+            (void)cudaGetLastError();
+            v = 1;
+        }
+        return v;
+    });
+    const int64_t slots = (int64_t)SMs * per_sm;
+    // the split (a cluster of at most 8, at least 4 steps each) with the
+    // fewest waves per unit of work: waves(S) / S, ties to the smaller S
+    int S = 1;
+    double best = 1e30;
+    for (int s = 1; s <= 8; ++s) {
+        if (s > 1 && K / (kSMStep * s) < 4) break;
+        const double cost = (double)((tiles * (int64_t)s + slots - 1) / slots) / s;
+        if (cost < best - 1e-9) {
+            best = cost;
+            S = s;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles, 1, S);
+    cfg.blockDim = dim3(kSMThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = S;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_f32_smallm_kernel<MT, TN>, A, W, absmax, bias, Y, M, N, K, log2B, tab);
+}
+
 size_t gemv_f32_smem(int K) {
     const size_t Kp = ((size_t)K + kVUnitK - 1) / kVUnitK * kVUnitK;
     return (16 * 32 + kVMaxRows + kVWarps * 8 + Kp) * sizeof(float);
@@ -346,6 +582,13 @@ cudaError_t launch_gemm_f32(const float *A, const uint8_t *W, const float *absma
     static const CodeTable nf4 = host_code_table(BNB4_NF4);
     static const CodeTable fp4 = host_code_table(BNB4_FP4);
     const CodeTable &tab = qt == BNB4_NF4 ? nf4 : fp4;
+    if (!backward && M <= 16) {
+        const int log2B_ = ilog2(blocksize);
+        const int m_ = (int)M, n_ = (int)N, k_ = (int)K;
+        if (M <= 4) return launch_smallm<4, 2>(A, W, absmax, bias, Y, m_, n_, k_, log2B_, tab, stream);
+        if (M <= 8) return launch_smallm<8, 2>(A, W, absmax, bias, Y, m_, n_, k_, log2B_, tab, stream);
+        return launch_smallm<16, 2>(A, W, absmax, bias, Y, m_, n_, k_, log2B_, tab, stream);
+    }
     const int ncols = (int)(backward ? K : N);
     const int log2B = ilog2(blocksize);
     // reduction split S (a cluster of S CTAs along z): enough CTAs for about

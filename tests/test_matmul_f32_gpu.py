@@ -112,3 +112,28 @@ def test_gemv_f32_decode_shapes_sampled(K, N):
                                 np.zeros(rows.size, np.int64), rows)
     absdot = np.abs(Wt.wdeq[rows].astype(np.float64)) @ np.abs(x.astype(np.float64)) + np.abs(b[rows])
     check(y[rows], ref, absdot, K)
+
+
+@pytest.mark.parametrize("K,N", [(8192, 28672), (28672, 8192)])
+def test_gemm_f32_small_m_70b_shapes_sampled(K, N):
+    """Llama-3-70B-shaped small-M projections in fp32 (NF4 B=64, bias), in the
+    launch the bench times: M = 4, 8 and 16, sampled output columns."""
+    w = synthetic.weight(N, K, 0, 0.015).numpy().reshape(-1)
+    packed, absmax = oracle.quantize(w, "f32", 64, "nf4")
+    del w
+    dp, da = torch.from_numpy(packed).cuda(), torch.from_numpy(absmax).cuda()
+    b = synthetic.bias(N, seed=2, dtype="f32").numpy()
+    cols = np.unique(np.concatenate([[0, N - 1], np.random.default_rng(N).integers(0, N, 126)]))
+    # the sampled rows of the exact fp32 weight, for the per-element bound
+    rb = K // 2
+    wsel = np.stack([oracle.dequantize(packed[c * rb:(c + 1) * rb], absmax[c * (K // 64):(c + 1) * (K // 64)],
+                                       K, 64, "nf4", "f32") for c in cols]).astype(np.float64)
+    for M in (4, 8, 16):
+        X = synthetic.activations(M, K, seed=M, dtype="f32").numpy()
+        Y = to_host(bnb4.gemm_4bit(to_dev(X.reshape(-1), "f32").view(M, K), dp, da, N,
+                                   to_dev(b, "f32"), 64, "nf4")).reshape(M, N)
+        ms = np.repeat(np.arange(M), cols.size)
+        ns = np.tile(cols, M)
+        ref = oracle.matmul_entries(X.reshape(-1), "f32", packed, absmax, b, M, N, K, 64, "nf4", ms, ns)
+        absdot = (np.abs(X.astype(np.float64)) @ np.abs(wsel).T + np.abs(b[cols])[None, :]).reshape(-1)
+        check(Y[ms, ns], ref, absdot, K)

@@ -627,9 +627,13 @@ def time_next_rows(step, dev, hbm):
         M = X.shape[0]
         X32 = X.float()
         Y32 = torch.empty(M, N, dtype=torch.float32, device=dev)
-        rec(f"gemm_4bit_f32_M{M}_{K}x{N}", graph_per_launch(dev, [
+        name = f"gemm_4bit_f32_M{M}_{K}x{N}"
+        rec(name, graph_per_launch(dev, [
             lambda i=i: b.gemm_4bit(X32, ps[i], as_[i], N, None, BLOCK, "nf4", out=Y32) for i in range(2)]),
             N * K // 2 + 4 * nb + 4 * M * K + 4 * M * N)
+        # at M = 16 the fp32 FMAs, not HBM, bound it: report both
+        tf = 2.0 * M * N * K / (out[name]["us"] / 1e6) / 1e12
+        out[name].update({"TFLOP/s": round(tf, 1), "fp32_fma_frac": round(tf / fp32_peak, 4)})
         del ps, as_
     M, K, N, p, a, X, dY, Y, dX = step.prefill
     X32, dY32 = X.float(), dY.float()

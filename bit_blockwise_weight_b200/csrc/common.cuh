@@ -151,6 +151,10 @@ QuantTables host_quant_tables(bnb4_quant_type qt);
 // q unusable, if a key cannot be placed.
 bool host_fp4_exact_tables(int p, QuantTables &q);
 
+// Screen tables for a code table whose thresholds every ratio of two p-bit
+// values stays clear of (NF4 with bf16 inputs), likewise exact (tables.cu).
+bool host_ratio_exact_tables(bnb4_quant_type qt, int p, QuantTables &q);
+
 // 12582925 = 1.5 * 2^23 + 13: the fma lands in [2^23, 2^24) where the fp32
 // spacing is 1, so the low mantissa bits hold rn(13 v + 13).
 __device__ __forceinline__ uint32_t cell_of(float v) {

@@ -1,7 +1,9 @@
 // tables.cu -- host construction of the code tables and of the decision
 // tables that the quantize kernel searches (see common.cuh).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <vector>
 #include <cstdlib>
 #include <cstring>
 
@@ -166,6 +168,75 @@ bool host_fp4_exact_tables(int p, QuantTables &q) {
         if (up ? !(Kd > T - gap + err && Kd < T - err) : !(Kd > T + err && Kd < T + gap - err)) return false;
         for (int j = 0; j <= 26; ++j)  // and the cell is still exact
             if (std::fabs(Kd - (j - 12.5) / 13.0) <= 0x1p-16) return false;
+        q.key[k] = kb;
+    }
+    return true;
+}
+
+// A table whose decision thresholds no ratio of two p-bit values comes near
+// (NF4 with bf16 inputs: every ratio x / a with |x| <= a lies at least 15 ulps
+// from every NF4 midpoint; fp16 ratios come within a fraction of an ulp, and
+// FP4's midpoints lie a fraction of an ulp from the ratios k / 24).  The ratios are enumerated (X / A 2^d: X < 2^p,
+// A in [2^(p-1), 2^p), d down to where no threshold is reached; a subnormal
+// absmax is outside the screen's range anyway); each key is put inside the
+// gap between the nearest ratios below and above its threshold, clear of
+// both by the screen's error with r = RN(1/a) (below |x / a| 2^-24), with the
+// rank nibble kept.  Returns false, leaving q unusable, where a gap is too
+// narrow.
+bool host_ratio_exact_tables(bnb4_quant_type qt, int p, QuantTables &q) {
+    q = host_quant_tables(qt);
+    if (!q.valid || q.fast == 0 || p < 2 || p > 11) return false;
+    const CodeTable c = host_code_table(qt);
+    std::vector<double> ratio;
+    ratio.reserve((size_t)1 << (2 * p - 1));
+    for (int A = 1 << (p - 1); A < (1 << p); ++A)
+        for (int X = 0; X < (1 << p); ++X) ratio.push_back((double)X / A);
+    std::sort(ratio.begin(), ratio.end());
+    for (int k = 0; k < 32; ++k) {
+        if (q.thr[k] == 2.0f) continue;  // no threshold in the cell
+        const int R = (int)((q.rank_lohi[k] >> 4) & 15u);
+        // the exact midpoint of the two codes the threshold separates
+        float lo_v = -2.0f, hi_v = 2.0f;
+        for (int i = 0; i < 16; ++i) {
+            if (c.v[i] <= q.thr[k] && c.v[i] > lo_v) lo_v = c.v[i];
+            if (c.v[i] > q.thr[k] && c.v[i] < hi_v) hi_v = c.v[i];
+        }
+        const double mid = 0.5 * ((double)lo_v + (double)hi_v), m = std::fabs(mid);
+        if (!(m > 0.0) || hi_v > 1.0f || lo_v < -1.0f) return false;
+        // nearest ratio magnitudes below and above |mid|, over the scalings
+        // that reach it (ratios below 2^-20 |mid| cannot)
+        double below = 0.0, above = 4.0;
+        for (int d = 1; d >= -40; --d) {
+            const double sc = std::ldexp(1.0, d);
+            if (2.0 * sc < m * 0x1p-20) break;
+            const double t = m / sc;
+            auto it = std::lower_bound(ratio.begin(), ratio.end(), t);
+            if (it != ratio.end()) {
+                if (*it == t) return false;  // a ratio on the midpoint
+                above = std::min(above, *it * sc);
+            }
+            if (it != ratio.begin()) below = std::max(below, *(it - 1) * sc);
+        }
+        // every ratio at least two ulps of the midpoint away, so its IEEE
+        // quotient (half an ulp off) falls on the same side of the threshold
+        // (within an ulp of the midpoint) as the ratio itself
+        const double u = std::ldexp(1.0, (int)std::floor(std::log2(m)) - 23);
+        if (m - below < 2 * u || above - m < 2 * u) return false;
+        const double err = above * 0x1p-24 * (1.0 + 0x1p-20) + 0x1p-60;
+        // the key (signed like the threshold) inside (below + err, above - err)
+        const double target = 0.5 * (below + above);
+        float K = (float)(mid < 0 ? -target : target);
+        uint32_t kb;
+        std::memcpy(&kb, &K, 4);
+        int64_t cand = (int64_t)((kb & ~15u) | (uint32_t)R);
+        if (cand - (int64_t)kb > 8) cand -= 16;
+        if ((int64_t)kb - cand > 8) cand += 16;
+        kb = (uint32_t)cand;
+        std::memcpy(&K, &kb, 4);
+        const double Km = std::fabs((double)K);
+        if (!(Km > below + err && Km < above - err)) return false;
+        for (int j = 0; j <= 26; ++j)  // and the cell is still exact
+            if (std::fabs((double)K - (j - 12.5) / 13.0) <= 0x1p-16) return false;
         q.key[k] = kb;
     }
     return true;

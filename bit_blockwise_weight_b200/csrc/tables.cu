@@ -153,7 +153,10 @@ bool host_fp4_exact_tables(int p, QuantTables &q) {
         const int e = (int)std::floor(std::log2(std::fabs(T)) - 1.0 - 1e-9) + 1;
         const double gap = std::ldexp(1.0, e - p) / 24.0;
         const double err = std::fabs(T) * 0x1p-24 * (1.0 + 0x1p-20) + 0x1p-60;
-        if (std::fabs(mid - T) > gap / 64) return false;
+        // the midpoint next to T, and the gap wide against an ulp, so a ratio
+        // a gap from T also has its IEEE quotient on its own side of thr
+        const double ulp = std::ldexp(1.0, (int)std::floor(std::log2(std::fabs(T))) - 23);
+        if (std::fabs(mid - T) > gap / 64 || gap < 16 * ulp) return false;
         float K = (float)(up ? T - gap / 2 : T + gap / 2);
         uint32_t kb;
         std::memcpy(&kb, &K, 4);
@@ -176,9 +179,10 @@ bool host_fp4_exact_tables(int p, QuantTables &q) {
 // A table whose decision thresholds no ratio of two p-bit values comes near
 // (NF4 with bf16 inputs: every ratio x / a with |x| <= a lies at least 15 ulps
 // from every NF4 midpoint; fp16 ratios come within a fraction of an ulp, and
-// FP4's midpoints lie a fraction of an ulp from the ratios k / 24).  The ratios are enumerated (X / A 2^d: X < 2^p,
-// A in [2^(p-1), 2^p), d down to where no threshold is reached; a subnormal
-// absmax is outside the screen's range anyway); each key is put inside the
+// FP4's midpoints lie a fraction of an ulp from the ratios k / 24).  The
+// ratios are enumerated (X / A 2^d: X < 2^p, A in [2^(p-1), 2^p), d down to
+// where no threshold is reached; a subnormal absmax is outside the screen's
+// range anyway); each key is put inside the
 // gap between the nearest ratios below and above its threshold, clear of
 // both by the screen's error with r = RN(1/a) (below |x / a| 2^-24), with the
 // rank nibble kept.  Returns false, leaving q unusable, where a gap is too

@@ -931,6 +931,7 @@ PROFILE_CASES = {
     "double_quant": "double_quant + dequant_absmax of 2^25 absmax values, groups of 256",
     "gemv_dq": "gemv_4bit_dq + bias, K=4096, N=14336, NF4 B=64, double-quantized absmax "
                "(groups of 256), bf16",
+    "gemm_f32_small": "gemm_4bit M=16, K=8192, N=28672, NF4 B=64, fp32",
 }
 
 
@@ -955,7 +956,8 @@ def profile_case(name):
         bnb4.dequant_absmax(q, s, 256)
     else:
         K, N, M = {"gemv": (4096, 14336, 1), "gemv_dq": (4096, 14336, 1), "gemm_small": (8192, 28672, 16),
-                   "gemm_tc": (4096, 14336, 512), "gemm_tc_backward": (4096, 14336, 512)}[name]
+                   "gemm_f32_small": (8192, 28672, 16), "gemm_tc": (4096, 14336, 512),
+                   "gemm_tc_backward": (4096, 14336, 512)}[name]
         w = synthetic.normal((N * K,), 0, 0.02, "f32", device=d)
         p, a = bnb4.quantize_4bit(w, BLOCK, "nf4")
         del w
@@ -966,6 +968,8 @@ def profile_case(name):
             q8, s8 = bnb4.double_quant(a, 256)
             bnb4.gemv_4bit_dq(synthetic.normal((K,), 1, 1.0, "bf16", device=d), p, q8, s8, N, K,
                               synthetic.normal((N,), 2, 1.0, "bf16", device=d))
+        elif name == "gemm_f32_small":
+            bnb4.gemm_4bit(synthetic.normal((M, K), 1, 1.0, "f32", device=d), p, a, N)
         elif name == "gemm_tc_backward":
             bnb4.gemm_4bit_backward(synthetic.normal((M, N), 3, 1.0, "bf16", device=d), p, a, K)
         else:
